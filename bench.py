@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""Throughput of the tiled, IO-aware attention path on B200.
+
+One step = one pass of the whole hot path over one synthetic batch: the
+forward (TMA-staged tiles, S = scale Q K^T, online softmax, PV, O/LSE
+epilogue) followed by the backward (D = rowsum(dO * O), dK/dV and dQ with P
+recomputed from LSE).  The workload is B=2, H=16, N=4096, d=128 (bf16),
+non-causal; causal and forward-only legs are reported beside it.
+
+Timing: W untimed warm-up steps, then K timed steps, each bracketed by CUDA
+events on the launching stream; a 256 MiB buffer is written between timed
+steps so that no step starts with its inputs in L2.  With N GPUs (torchrun,
+one rank per GPU) every rank runs its own independent batch (weak scaling,
+no collective on the data path); rank 0 prints the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other place this
+script runs it) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+_ROOT = os.path.dirname(os.path.abspath(__file__))
+if _ROOT not in sys.path:
+    sys.path.insert(0, _ROOT)
+
+METRIC = "attention TFLOP/s fwd & fwd+bwd (bf16, N=4096, d=128) and % of BF16 tensor peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "fwd_b2h16n4096d128"
+
+
+def _peaks():
+    p = os.path.join(_ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def _flops(B, H, N, d, causal):
+    fwd = 4.0 * B * H * N * N * d
+    if causal:
+        fwd /= 2
+    return fwd, 2.5 * fwd
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle as a baseline (bounded sample)
+# ---------------------------------------------------------------------------
+def oracle_sample_run(N=4096, d=128, causal=False, heads=1, seed=0):
+    """fwd + bwd of `heads` heads of the workload in fp64 on the host cores.
+    Returns (seconds, flops by the same convention as the GPU number)."""
+    import oracle
+    from io_aware_tiled_b200.inputs import attention_inputs
+    q, k, v, do = attention_inputs(1, heads, N, d, seed=seed)
+    args = [t.double().numpy() for t in (q, k, v, do)]
+    t0 = time.perf_counter()
+    oracle.backward(*args, causal, 1.0 / math.sqrt(d))
+    dt = time.perf_counter() - t0
+    f, b = _flops(1, heads, N, d, causal)
+    return dt, f + b
+
+
+def cpu_baseline(target_s=12.0):
+    import oracle
+    total_t, total_f, reps = 0.0, 0.0, 0
+    while total_t < target_s and reps < 8:
+        dt, fl = oracle_sample_run()
+        total_t += dt
+        total_f += fl
+        reps += 1
+    return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} x one head (B=1,H=1,N=4096,d=128) fwd+bwd non-causal, fp64, {total_t:.1f} s",
+            "host_cpu_count": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    for _ in range(args.warmup):
+        oracle_sample_run()
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample_run()
+        times.append(dt)
+        flops += fl
+    total = sum(times)
+    value = flops / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": 2, "H": 16, "N": 4096, "d": 128, "causal": False,
+                   "step": "fwd+bwd", "sample": "one head per step (B=1,H=1,N=4096,d=128)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": "one head (B=1,H=1,N=4096,d=128) fwd+bwd non-causal per step, fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from io_aware_tiled_b200 import fa
+    from io_aware_tiled_b200.configs import WORKLOADS
+    from io_aware_tiled_b200.inputs import attention_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[WORKLOAD]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    q, k, v, do = attention_inputs(B, H, N, d, seed=w.seed + rank)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+    ws = torch.empty(fa.workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd(causal):
+        fa.forward(qd, kd, vd, causal, out=o, lse=lse)
+
+    def bwd(causal):
+        fa.backward(qd, kd, vd, o, dod, lse, causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, steps, per_kernel=False):
+        """Run fn `steps` times, L2 flushed before each; returns total ms and
+        per-kernel ms lists when per_kernel (forward + the three backward kernels)."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        kev = []
+        barrier()
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            if per_kernel:
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+                e[0].record(stream)
+                fwd(False)
+                fa.set_backward_phase_events(e[1:5])
+                bwd(False)
+                fa.set_backward_phase_events(None)
+                kev.append(e)
+            else:
+                fn()
+            ev[i][1].record(stream)
+        barrier()
+        total = sum(a.elapsed_time(b) for a, b in ev)
+        kern = None
+        if per_kernel:
+            kern = {"fa_fwd_kernel": [e[0].elapsed_time(e[1]) for e in kev],
+                    "fa_bwd_preprocess_kernel": [e[1].elapsed_time(e[2]) for e in kev],
+                    "fa_bwd_dkdv_kernel": [e[2].elapsed_time(e[3]) for e in kev],
+                    "fa_bwd_dq_kernel": [e[3].elapsed_time(e[4]) for e in kev]}
+        return total, kern
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (also the status check: a kernel timeout would show here)
+    for _ in range(max(args.warmup, 3)):
+        fwd(False); bwd(False); fwd(True); bwd(True)
+    rc = fa.sync_status(dev)
+    if rc != fa.FA_OK:
+        raise RuntimeError(f"library status {fa.status_string(rc)}")
+
+    f_nc, b_nc = _flops(B, H, N, d, False)
+    f_c, b_c = _flops(B, H, N, d, True)
+
+    clocks = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    with clocks:
+        main_ms, kern = timed(None, args.steps, per_kernel=True)
+        fwd_ms, _ = timed(lambda: fwd(False), args.steps)
+        fwdc_ms, _ = timed(lambda: fwd(True), args.steps)
+        stepc_ms, _ = timed(lambda: (fwd(True), bwd(True)), args.steps)
+    main_ms = max_over_ranks(main_ms)
+    fwd_ms = max_over_ranks(fwd_ms)
+    fwdc_ms = max_over_ranks(fwdc_ms)
+    stepc_ms = max_over_ranks(stepc_ms)
+    rc = fa.sync_status(dev)
+    if rc != fa.FA_OK:
+        raise RuntimeError(f"library status {fa.status_string(rc)}")
+
+    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host
+    hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+    ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
+    hl = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q2, k2, v2, do2 = (t.to(dev, non_blocking=True) for t in (hq, hk, hv, hdo))
+        o2, l2 = fa.forward(q2, k2, v2, False)
+        g = fa.backward(q2, k2, v2, o2, do2, l2, False, workspace=ws)
+        for h, t in zip((ho, hl, hdq, hdk, hdv), (o2, l2, *g)):
+            h.copy_(t, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms, _ = timed(e2e_step, max(3, args.steps // 4))
+    e2e_steps = max(3, args.steps // 4)
+    e2e_ms = max_over_ranks(e2e_ms)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
+
+    peaks = _peaks()
+    step_flops = f_nc + b_nc
+    value = world * step_flops * args.steps / (main_ms * 1e-3) / 1e12
+    # per-kernel live durations (rank-local) and the dominant kernel's roofline
+    kavg = {n: sum(v) / len(v) for n, v in kern.items()}
+    per_kernel_flops = {  # dense MMA work each kernel performs
+        "fa_fwd_kernel": 4.0 * B * H * N * N * d,
+        "fa_bwd_dkdv_kernel": 8.0 * B * H * N * N * d,   # S^T, dP^T, dV, dK
+        "fa_bwd_dq_kernel": 6.0 * B * H * N * N * d,     # S, dP, dQ
+    }
+    dom = max(kavg, key=kavg.get)
+    peak = peaks["bf16_tflops"]
+    if dom in per_kernel_flops:
+        ach = per_kernel_flops[dom] / (kavg[dom] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": None, "peak_kind": f"bf16 burst, {peaks['source']}"}
+    else:
+        bytes_pre = 2.0 * B * H * N * d * 2 + 4.0 * B * H * N
+        ach = bytes_pre / (kavg[dom] * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_kind": f"hbm copy, {peaks['source']}"}
+    kernels = {n: {"ms": kavg[n],
+                   "tflops": (per_kernel_flops[n] / (kavg[n] * 1e-3) / 1e12) if n in per_kernel_flops else None}
+               for n in kavg}
+    kernels["fa_bwd_preprocess_kernel"]["gbs"] = (2.0 * B * H * N * d * 2 + 4.0 * B * H * N) / (
+        kavg["fa_bwd_preprocess_kernel"] * 1e-3) / 1e9
+
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": d, "causal": False, "step": "fwd+bwd",
+                       "inputs": "i.i.d. N(0,1) bf16 from seed 0 (+rank)", "l2": "256 MiB written between timed steps",
+                       "parallelism": f"independent batch per GPU x{world}"},
+            "frac_of_peak": value / peak,
+            "legs": {
+                "fwd_noncausal": {"tflops": world * f_nc * args.steps / (fwd_ms * 1e-3) / 1e12,
+                                  "ms": fwd_ms / args.steps},
+                "fwd_causal": {"tflops": world * f_c * args.steps / (fwdc_ms * 1e-3) / 1e12,
+                               "ms": fwdc_ms / args.steps},
+                "fwd_bwd_causal": {"tflops": world * (f_c + b_c) * args.steps / (stepc_ms * 1e-3) / 1e12,
+                                   "ms": stepc_ms / args.steps},
+            },
+            "kernels": kernels,
+            "roofline": roof,
+            "e2e": {"value": world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks.summary(),
+            "peaks": peaks,
+        }
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=__import__("torch").device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

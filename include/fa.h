@@ -1,0 +1,125 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) tiled, IO-aware exact attention library (libfa.so).
+ *
+ * The operation is exact scaled-dot-product attention
+ *     S = scale * Q K^T,  P = softmax(S) row by row,  O = P V,
+ * computed tile by tile with an online softmax so that the N x N matrices S
+ * and P never reach device memory ("FlashAttention分块计算优化Transformer显存
+ * 效率", section 1.1 for the problem and the tiled loop, section 3.2 for the
+ * online softmax, section 2.2 for causal block skipping).  The backward pass
+ * keeps only O and one statistic per row and recomputes P tile by tile
+ * ("图解Flash Attention运算原理", 总结: Recomputation).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors Q, K, V, O, dO, dQ, dK, dV: bf16, shape [B, H, N, d], contiguous
+ *    row-major (d fastest), in device memory of the current CUDA device.
+ *  - LSE: fp32 [B, H, N]; LSE[b,h,i] = ln sum_j exp(S_ij), the natural-log
+ *    logsumexp of row i of the SCALED, masked scores.
+ *  - d must be 64 or 128; B, H, N must be positive (a non-positive size is
+ *    rejected, as the capacity model of "14. FlashAttention Memory Model"
+ *    rejects non-positive sizes); B*H*N must fit in a 32-bit signed int.
+ *  - causal != 0 applies the lower-triangular mask: key j is visible to query
+ *    i iff j <= i.  Fully masked key tiles are skipped, not computed.
+ *  - scale: finite; a value <= 0 selects 1/sqrt(d).
+ *  - Every pointer must be non-null and 16-byte aligned.  Outputs must not
+ *    overlap inputs or each other.
+ *  - stream: a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Calls are asynchronous: they validate, enqueue and return.  Validation
+ *    and launch failures are returned synchronously and nothing is written.
+ *    A stall inside a kernel (every internal wait has a wall-clock limit of
+ *    2 s) is reported by fa_sync_status as FA_ERR_TIMEOUT.
+ *  - Ownership: the caller owns every buffer, including the backward
+ *    workspace.  The library allocates no device memory and keeps no state
+ *    between calls except per-device attribute caches and the device error
+ *    word read by fa_sync_status.
+ *  - Device: NVIDIA B200 class (compute capability 10.0, sm_100a) only.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1,        /* null pointer, bad size, d not in {64,128}, bad scale, overlap */
+  FA_ERR_ALIGNMENT = -2,          /* a pointer is not 16-byte aligned */
+  FA_ERR_UNSUPPORTED_DEVICE = -3, /* current device is not sm_100, or a pointer is not device memory */
+  FA_ERR_LAUNCH = -4,             /* a CUDA call or kernel launch failed */
+  FA_ERR_WORKSPACE = -5,          /* backward workspace missing, misaligned or too small */
+  FA_ERR_TIMEOUT = -6             /* a kernel's internal wait ran out (reported by fa_sync_status) */
+} fa_status;
+
+/*
+ * Forward pass.
+ * In:  Q, K, V [B,H,N,d] bf16.
+ * Out: O [B,H,N,d] bf16 (O = P V, rounded to nearest even), LSE [B,H,N] fp32.
+ * One persistent kernel launch on `stream`.
+ * Returns FA_OK or an fa_status error code (nothing written on error).
+ */
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+           int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes (the fp32 row
+ * vector D = rowsum(dO * O), [B,H,N], rounded up to 256 bytes).  Returns 0
+ * for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass for the loss L = sum(dO * O).
+ * In:  Q, K, V, O (the forward's output), dO [B,H,N,d] bf16; LSE [B,H,N] fp32
+ *      from fa_fwd with the same causal flag and scale.
+ * Out: dQ, dK, dV [B,H,N,d] bf16.
+ * Workspace: caller-owned device buffer of at least fa_bwd_workspace_bytes()
+ *      bytes, 16-byte aligned; its contents on entry do not matter.
+ * Launches, in order on `stream`: the D = rowsum(dO * O) pass, the dK/dV
+ * kernel, the dQ kernel.  P is recomputed as exp(S - LSE).
+ */
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+           void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
+           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reports: FA_ERR_LAUNCH if a CUDA error is
+ * pending, FA_ERR_TIMEOUT if a kernel of this library recorded a wait
+ * timeout since the last call (the record is then cleared), else FA_OK.
+ */
+int fa_sync_status(void* stream);
+
+/*
+ * The raw device error word recorded with the last FA_ERR_TIMEOUT reported
+ * by fa_sync_status ((wait site << 8) | code; 0 if none).  For diagnosis.
+ */
+unsigned int fa_last_error_word(void);
+
+/*
+ * Optional per-kernel timing of fa_bwd (profiling aid).  When set, fa_bwd
+ * records the four cudaEvent_t handles (passed as void*) on its stream:
+ * e0 before the D pass, e1 before the dK/dV kernel, e2 before the dQ
+ * kernel, e3 after it.  Events belong to the caller and must stay valid while
+ * set; pass four NULLs to stop.  The setting is process-wide.
+ */
+void fa_bwd_set_phase_events(void* e0, void* e1, void* e2, void* e3);
+
+/* Human-readable name of an fa_status value (static string). */
+const char* fa_status_string(int status);
+
+/*
+ * Fault-detection self test.  Launches one tiny kernel that waits on a
+ * barrier nothing ever signals, with a wall-clock limit of `limit_us`
+ * microseconds (1 .. 10,000,000).  The wait runs out, the kernel records
+ * FA_ERR_TIMEOUT and returns; the next fa_sync_status(stream) reports it and
+ * the CUDA context stays usable.  Nothing faults or traps.
+ */
+int fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,335 @@
+// fa_api.cu -- the C ABI of libfa.so: argument validation, TMA descriptor
+// encoding and kernel launches for the sm_100a attention kernels.
+#include <math.h>
+#include <mutex>
+#include <stdint.h>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D view [BH][N][d] of a bf16 [B,H,N,d] tensor; box = 64 columns x box_rows
+// rows x 1 head, 128-byte swizzle.  Rows past N read as zero within the head.
+bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int checked = 0;  // 0 unknown, 1 supported, -1 unsupported
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+template <typename Kern>
+bool set_smem(Kern k, int bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// Returns FA_OK and the SM count if the current device is sm_100 and the
+// kernels' shared-memory limits are set on it.
+int device_ready(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_UNSUPPORTED_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (di.checked == 0) {
+    int major = 0, minor = 0, n = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    bool ok = (major == 10 && minor == 0) && n > 0;
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, false>, fa::FwdCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, true>, fa::FwdCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, false>, fa::FwdCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, true>, fa::FwdCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<64, false>, fa::DkdvCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<64, true>, fa::DkdvCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<128, false>, fa::DkdvCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<128, true>, fa::DkdvCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dq_kernel<64, false>, fa::DqCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dq_kernel<64, true>, fa::DqCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, false>, fa::DqCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, true>, fa::DqCfg<128>::SMEM_BYTES);
+    cudaGetLastError();
+    di.checked = ok ? 1 : -1;
+    di.sms = n;
+  }
+  if (di.checked != 1) return FA_ERR_UNSUPPORTED_DEVICE;
+  *sms = di.sms;
+  return FA_OK;
+}
+
+cudaEvent_t g_phase_events[4] = {nullptr, nullptr, nullptr, nullptr};
+std::mutex g_events_mu;
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+int check_sizes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+float effective_scale(float scale, int d, bool* ok) {
+  *ok = isfinite(scale);
+  return scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(d));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_UNSUPPORTED_DEVICE: return "FA_ERR_UNSUPPORTED_DEVICE";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+           int causal, float scale, void* stream) {
+  int rc = check_sizes(B, H, N, d);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FA_ERR_ALIGNMENT;
+  bool scale_ok = false;
+  const float sc = effective_scale(scale, d, &scale_ok);
+  if (!scale_ok) return FA_ERR_INVALID_ARG;
+  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2, lbytes = static_cast<size_t>(B) * H * N * 4;
+  const Range rq{(uintptr_t)Q, (uintptr_t)Q + tbytes}, rk{(uintptr_t)K, (uintptr_t)K + tbytes},
+      rv{(uintptr_t)V, (uintptr_t)V + tbytes}, ro{(uintptr_t)O, (uintptr_t)O + tbytes},
+      rl{(uintptr_t)LSE, (uintptr_t)LSE + lbytes};
+  if (overlaps(ro, rq) || overlaps(ro, rk) || overlaps(ro, rv) || overlaps(ro, rl) || overlaps(rl, rq) ||
+      overlaps(rl, rk) || overlaps(rl, rv))
+    return FA_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((rc = device_ready(&sms))) return rc;
+  if (!is_device_ptr(Q) || !is_device_ptr(K) || !is_device_ptr(V) || !is_device_ptr(O) || !is_device_ptr(LSE))
+    return FA_ERR_UNSUPPORTED_DEVICE;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, BH, N, d, 128) || !make_map(&mk, K, BH, N, d, 128) || !make_map(&mv, V, BH, N, d, 128))
+    return FA_ERR_LAUNCH;
+  const int nqt = (N + 127) / 128, units = BH * ((nqt + 1) / 2);
+  const int grid = units < sms ? units : sms;
+  const float sl2 = sc * fa::kLog2e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* o = static_cast<__nv_bfloat16*>(O);
+  if (d == 64) {
+    if (causal) fa::fa_fwd_kernel<64, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+    else fa::fa_fwd_kernel<64, false><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+  } else {
+    if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+    else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d)) return 0;
+  const size_t dbytes = static_cast<size_t>(B) * H * N * 4;
+  return (dbytes + 255) & ~static_cast<size_t>(255);
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, d);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return FA_ERR_ALIGNMENT;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d))
+    return FA_ERR_WORKSPACE;
+  bool scale_ok = false;
+  const float sc = effective_scale(scale, d, &scale_ok);
+  if (!scale_ok) return FA_ERR_INVALID_ARG;
+  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2, lbytes = static_cast<size_t>(B) * H * N * 4;
+  const Range ins[6] = {{(uintptr_t)Q, (uintptr_t)Q + tbytes},   {(uintptr_t)K, (uintptr_t)K + tbytes},
+                        {(uintptr_t)V, (uintptr_t)V + tbytes},   {(uintptr_t)O, (uintptr_t)O + tbytes},
+                        {(uintptr_t)dO, (uintptr_t)dO + tbytes}, {(uintptr_t)LSE, (uintptr_t)LSE + lbytes}};
+  const Range outs[4] = {{(uintptr_t)dQ, (uintptr_t)dQ + tbytes},
+                         {(uintptr_t)dK, (uintptr_t)dK + tbytes},
+                         {(uintptr_t)dV, (uintptr_t)dV + tbytes},
+                         {(uintptr_t)workspace, (uintptr_t)workspace + fa_bwd_workspace_bytes(B, H, N, d)}};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], ins[b])) return a == 3 ? FA_ERR_WORKSPACE : FA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], outs[b])) return b == 3 ? FA_ERR_WORKSPACE : FA_ERR_INVALID_ARG;
+  }
+  int sms = 0;
+  if ((rc = device_ready(&sms))) return rc;
+  const void* ptrs[10] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
+  for (const void* p : ptrs)
+    if (!is_device_ptr(p)) return FA_ERR_UNSUPPORTED_DEVICE;
+  const int BH = B * H;
+  CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128, mk64, mv64;
+  if (!make_map(&mq64, Q, BH, N, d, 64) || !make_map(&mdo64, dO, BH, N, d, 64) ||
+      !make_map(&mk128, K, BH, N, d, 128) || !make_map(&mv128, V, BH, N, d, 128) ||
+      !make_map(&mq128, Q, BH, N, d, 128) || !make_map(&mdo128, dO, BH, N, d, 128) ||
+      !make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64))
+    return FA_ERR_LAUNCH;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* Dvec = static_cast<float*>(workspace);
+  const long long rows = static_cast<long long>(BH) * N;
+  const float sl2 = sc * fa::kLog2e;
+  auto* dq = static_cast<__nv_bfloat16*>(dQ);
+  auto* dk = static_cast<__nv_bfloat16*>(dK);
+  auto* dv = static_cast<__nv_bfloat16*>(dV);
+  auto* o = static_cast<const __nv_bfloat16*>(O);
+  auto* dob = static_cast<const __nv_bfloat16*>(dO);
+  cudaEvent_t ev[4];
+  {
+    std::lock_guard<std::mutex> lock(g_events_mu);
+    for (int e = 0; e < 4; ++e) ev[e] = g_phase_events[e];
+  }
+  auto mark = [&](int e) {
+    if (ev[e]) cudaEventRecord(ev[e], s);
+  };
+  const int grid_kv = BH * ((N + 127) / 128);
+  const int grid_q = BH * ((N + 127) / 128);
+  if (d == 64) {
+    const long long threads = rows * 8;
+    mark(0);
+    fa::fa_bwd_preprocess_kernel<64><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(o, dob, Dvec, rows);
+    mark(1);
+    if (causal) {
+      fa::fa_bwd_dkdv_kernel<64, true><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      mark(2);
+      fa::fa_bwd_dq_kernel<64, true><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
+      mark(3);
+    } else {
+      fa::fa_bwd_dkdv_kernel<64, false><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      mark(2);
+      fa::fa_bwd_dq_kernel<64, false><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
+      mark(3);
+    }
+  } else {
+    const long long threads = rows * 16;
+    mark(0);
+    fa::fa_bwd_preprocess_kernel<128><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(o, dob, Dvec, rows);
+    mark(1);
+    if (causal) {
+      fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      mark(2);
+      fa::fa_bwd_dq_kernel<128, true><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
+      mark(3);
+    } else {
+      fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      mark(2);
+      fa::fa_bwd_dq_kernel<128, false><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
+      mark(3);
+    }
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+static unsigned int g_last_error_word = 0;
+
+void fa_bwd_set_phase_events(void* e0, void* e1, void* e2, void* e3) {
+  std::lock_guard<std::mutex> lock(g_events_mu);
+  g_phase_events[0] = static_cast<cudaEvent_t>(e0);
+  g_phase_events[1] = static_cast<cudaEvent_t>(e1);
+  g_phase_events[2] = static_cast<cudaEvent_t>(e2);
+  g_phase_events[3] = static_cast<cudaEvent_t>(e3);
+}
+
+int fa_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_error_word, sizeof(word)) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    g_last_error_word = word;
+    if (cudaMemcpyToSymbol(fa::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_LAUNCH;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+unsigned int fa_last_error_word(void) { return g_last_error_word; }
+
+}  // extern "C"
+
+namespace fa {
+// One warp initialises a barrier that nothing arrives on and waits for it
+// with a short wall-clock limit; the wait records the timeout and returns.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait_slow(b, 0, 255u, limit_ns);
+}
+}  // namespace fa
+
+extern "C" int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 10000000u) return FA_ERR_INVALID_ARG;
+  int sms = 0;
+  int rc = device_ready(&sms);
+  if (rc) return rc;
+  fa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}

@@ -1,0 +1,387 @@
+// fa_fwd.cuh -- forward kernel of tiled, IO-aware exact attention for sm_100a.
+//
+// What it computes (per head, per query row i):
+//   S_ij = scale * q_i . k_j, masked (causal: j > i; ragged tail: j >= N),
+//   O_i  = sum_j softmax(S_i)_j v_j,   LSE_i = ln sum_j exp(S_ij),
+// tile by tile, so the N x N S and P never leave the SM
+// ("FlashAttention分块计算优化Transformer显存效率", section 1.1 tiled loop;
+// section 3.2 online softmax: running max m, running sum l, the partial O
+// rescaled by exp(m_old - m_new); section 2.2 causal block skipping with
+// masking only on the diagonal blocks).  The final O = O_partial / l and the
+// stored statistic LSE = m + ln l are the completion of section 3.2 that makes
+// the result equal the global softmax ("图解Flash Attention运算原理", 分块 Softmax).
+//
+// B200 design (what differs from the pages' A100-era sizing):
+//   * One persistent CTA per SM; a work unit is a PAIR of 128-row Q tiles of
+//     one (batch, head).  Two softmax warpgroups (one per Q tile) alternate, so
+//     the tensor core computes one tile's S or PV while the other tile's
+//     exponentials run.
+//   * Three warpgroups: the control warpgroup gives registers back
+//     (setmaxnreg) to the two softmax warpgroups, which hold a full S row each.
+//   * Warp 0 issues TMA loads: Q pair once per unit, K_j and V_j through
+//     separate rings of ST stages (128 keys x d, 128-byte swizzle).
+//   * Warp 1 issues tcgen05.mma from one thread: S_t = Q_t K_j^T (M=128,
+//     N=128, K=d, both operands K-major in shared memory) into tensor memory,
+//     and O_t += P_t V_j (M=128, N=d, K=128) with P_t read from TENSOR MEMORY
+//     (bf16, written over S_t's columns) and V_j MN-major from shared memory.
+//   * Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1
+//     [128,256), O0 [256, 256+d), O1 [256+d, 256+2d).
+//   * Softmax: each thread owns one full row of S (tcgen05.ld 32x32b), so the
+//     row max and row sum are register reductions.  Work is in base 2 with
+//     scale*log2(e) folded into one FMA.  O is rescaled only when a row's max
+//     grows by more than 2^8 (exact: the final division uses the same max).
+//   * Epilogue: O / l as bf16 and LSE as fp32, stored once per row.
+#pragma once
+
+#include "fa_device.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;                 // query rows per Q tile
+  static constexpr int BN = 128;                 // keys per K/V tile
+  static constexpr int CH = D / 64;              // 128-byte column chunks per row
+  static constexpr int CHUNK = 128 * 128;        // bytes of one 64-column chunk of a 128-row tile
+  static constexpr int Q_TILE = BM * D * 2;
+  static constexpr int KV_TILE = BN * D * 2;
+  static constexpr int ST = (D == 128) ? 2 : 4;  // K and V ring depth
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_V = OFF_K + ST * KV_TILE;
+  static constexpr int OFF_BAR = OFF_V + ST * KV_TILE;
+  // barrier indices
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
+  static constexpr int B_K_FULL = 2, B_K_EMPTY = 2 + ST, B_V_FULL = 2 + 2 * ST, B_V_EMPTY = 2 + 3 * ST;
+  static constexpr int B_S_FULL = 2 + 4 * ST, B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2,
+                       B_O_EMPTY = B_O_FULL + 2;
+  static constexpr int NUM_BARS = B_O_EMPTY + 2;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;  // + room to align the base to 1024
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 idle; warpgroups 1 and 2: softmax of Q tile 0 and 1
+  static constexpr int THREADS = 384;
+  // register split (launch: 384 threads x 168): control warpgroup 56, softmax warpgroups 216 each
+  static constexpr uint32_t REGS_CONTROL = 56, REGS_SOFTMAX = 216;
+  static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+};
+
+// wait-site identifiers recorded in the error word
+enum FwdWaitSite : unsigned int {
+  FW_PROD_Q = 1, FW_PROD_K, FW_PROD_V, FW_MMA_Q, FW_MMA_K, FW_MMA_V, FW_MMA_P, FW_MMA_OE, FW_SM_S, FW_SM_O
+};
+
+__device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool causal, int& bh, int& qp) {
+  const int r = u / BH;
+  bh = u - r * BH;
+  qp = causal ? (NP - 1 - r) : r;  // causal: longest units first
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
+                  float* __restrict__ LSE, int BH, int N, float scale_log2) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
+  const uint32_t bars = sbase + C::OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars + 8 * C::B_Q_FULL, 1);
+    mbar_init(bars + 8 * C::B_Q_EMPTY, 1);
+    for (int s = 0; s < C::ST; ++s) {
+      mbar_init(bars + 8 * (C::B_K_FULL + s), 1);
+      mbar_init(bars + 8 * (C::B_K_EMPTY + s), 1);
+      mbar_init(bars + 8 * (C::B_V_FULL + s), 1);
+      mbar_init(bars + 8 * (C::B_V_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bars + 8 * (C::B_S_FULL + t), 1);
+      mbar_init(bars + 8 * (C::B_P_FULL + t), 128);
+      mbar_init(bars + 8 * (C::B_O_FULL + t), 1);
+      mbar_init(bars + 8 * (C::B_O_EMPTY + t), 128);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int NKT = (N + C::BN - 1) / C::BN;  // key tiles
+  const int NQT = (N + C::BM - 1) / C::BM;  // query tiles
+  const int NP = (NQT + 1) / 2;             // query tile pairs
+  const int units = BH * NP;
+
+  // Each role's setmaxnreg dominates that role's code, and the paths join only
+  // at the teardown, so the compiler gives each region its own register limit.
+  if (warp < 4) {
+    regs_dec<C::REGS_CONTROL>();
+    if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_it = 0, q_it = 0;
+      for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        int bh, qp;
+        fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
+        const int nk1 = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
+        if (!mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it & 1) ^ 1, FW_PROD_Q)) break;
+        ++q_it;
+        mbar_arrive_expect_tx(bars + 8 * C::B_Q_FULL, 2 * C::Q_TILE);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(sQ + t * C::Q_TILE + c * C::CHUNK, &tmQ, bars + 8 * C::B_Q_FULL, c * 64,
+                        (2 * qp + t) * C::BM, bh);
+        bool ok = true;
+        for (int j = 0; j < nk1; ++j, ++kv_it) {
+          const int s = kv_it % C::ST;
+          const uint32_t ph = (kv_it / C::ST) & 1;
+          if (!mbar_wait(bars + 8 * (C::B_K_EMPTY + s), ph ^ 1, FW_PROD_K)) { ok = false; break; }
+          mbar_arrive_expect_tx(bars + 8 * (C::B_K_FULL + s), C::KV_TILE);
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(sK + s * C::KV_TILE + c * C::CHUNK, &tmK, bars + 8 * (C::B_K_FULL + s), c * 64,
+                        j * C::BN, bh);
+          if (!mbar_wait(bars + 8 * (C::B_V_EMPTY + s), ph ^ 1, FW_PROD_V)) { ok = false; break; }
+          mbar_arrive_expect_tx(bars + 8 * (C::B_V_FULL + s), C::KV_TILE);
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(sV + s * C::KV_TILE + c * C::CHUNK, &tmV, bars + 8 * (C::B_V_FULL + s), c * 64,
+                        j * C::BN, bh);
+        }
+        if (!ok) break;
+      }
+    }
+    } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
+      // S = Q_t K_j^T: D/16 steps of K = 16 (32 bytes inside a 128-byte row; the
+      // next 64-column chunk starts CHUNK bytes later).
+      auto issue_s = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+        const uint32_t hi = sdesc_hi(1024);
+#pragma unroll 1
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          mma_ss(d_tmem, sdesc_make(sdesc_lo(a_smem + off, 16), hi), sdesc_make(sdesc_lo(b_smem + off, 16), hi),
+                 IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P_t V_j: 8 steps of 16 keys; P_t from tensor memory (8 columns of
+      // packed bf16 per step), V_j MN-major (16 rows of 128 bytes per step).
+      auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
+        const uint32_t hi = sdesc_hi(1024);
+#pragma unroll 1
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_ts(d_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_smem + kk * 16 * 128, C::CHUNK), hi), IDESC_PV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      uint32_t kv_it = 0, q_it = 0, unit_it = 0;
+      uint32_t p_ph0 = 0, p_ph1 = 0;
+      for (int u = blockIdx.x; u < units; u += gridDim.x, ++unit_it) {
+        int bh, qp;
+        fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
+        (void)bh;
+        const int nk0 = CAUSAL ? min(2 * qp + 1, NKT) : NKT;
+        const int nk1 = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
+        bool ok = mbar_wait(bars + 8 * C::B_Q_FULL, q_it & 1, FW_MMA_Q);
+        ++q_it;
+        if (!ok) break;
+        tc_fence_after();
+        {
+          const int s = kv_it % C::ST;
+          if (!mbar_wait(bars + 8 * (C::B_K_FULL + s), (kv_it / C::ST) & 1, FW_MMA_K)) break;
+          tc_fence_after();
+          issue_s(tmem + C::TM_S0, sQ, sK + s * C::KV_TILE);
+          tc_commit(bars + 8 * (C::B_S_FULL + 0));
+          issue_s(tmem + C::TM_S1, sQ + C::Q_TILE, sK + s * C::KV_TILE);
+          tc_commit(bars + 8 * (C::B_S_FULL + 1));
+          tc_commit(bars + 8 * (C::B_K_EMPTY + s));
+        }
+        for (int j = 0; j < nk1 && ok; ++j) {
+          const uint32_t it = kv_it + j;
+          const int s = it % C::ST;
+          if (!(ok = mbar_wait(bars + 8 * (C::B_V_FULL + s), (it / C::ST) & 1, FW_MMA_V))) break;
+          tc_fence_after();
+          if (j < nk0) {
+            if (!(ok = mbar_wait(bars + 8 * (C::B_P_FULL + 0), p_ph0, FW_MMA_P))) break;
+            p_ph0 ^= 1;
+            if (j == 0 && !(ok = mbar_wait(bars + 8 * (C::B_O_EMPTY + 0), (unit_it & 1) ^ 1, FW_MMA_OE))) break;
+            tc_fence_after();
+            issue_pv(tmem + C::TM_O0, tmem + C::TM_S0, sV + s * C::KV_TILE, j > 0);
+            if (j == nk0 - 1) tc_commit(bars + 8 * (C::B_O_FULL + 0));
+          }
+          const bool more = j + 1 < nk1;
+          const int sn = (it + 1) % C::ST;
+          if (more) {
+            if (!(ok = mbar_wait(bars + 8 * (C::B_K_FULL + sn), ((it + 1) / C::ST) & 1, FW_MMA_K))) break;
+            tc_fence_after();
+            if (j + 1 < nk0) {
+              issue_s(tmem + C::TM_S0, sQ, sK + sn * C::KV_TILE);
+              tc_commit(bars + 8 * (C::B_S_FULL + 0));
+            }
+          }
+          if (!(ok = mbar_wait(bars + 8 * (C::B_P_FULL + 1), p_ph1, FW_MMA_P))) break;
+          p_ph1 ^= 1;
+          if (j == 0 && !(ok = mbar_wait(bars + 8 * (C::B_O_EMPTY + 1), (unit_it & 1) ^ 1, FW_MMA_OE))) break;
+          tc_fence_after();
+          issue_pv(tmem + C::TM_O1, tmem + C::TM_S1, sV + s * C::KV_TILE, j > 0);
+          tc_commit(bars + 8 * (C::B_V_EMPTY + s));
+          if (j == nk1 - 1) tc_commit(bars + 8 * (C::B_O_FULL + 1));
+          if (more) {
+            issue_s(tmem + C::TM_S1, sQ + C::Q_TILE, sK + sn * C::KV_TILE);
+            tc_commit(bars + 8 * (C::B_S_FULL + 1));
+            tc_commit(bars + 8 * (C::B_K_EMPTY + sn));
+          }
+        }
+        if (!ok) break;
+        tc_commit(bars + 8 * C::B_Q_EMPTY);
+        kv_it += nk1;
+      }
+      // The last unit's Q_EMPTY arrival is the last one this thread's commits
+      // make; wait for it so no arrival lands after the CTA has exited.
+      if (q_it > 0) mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it - 1) & 1, FW_MMA_Q);
+    }
+    }
+    // teardown (each branch has its own, so the register regions never merge)
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+  } else {
+    regs_inc<C::REGS_SOFTMAX>();
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 4) >> 2;          // which Q tile of the pair
+    const int sp = warp & 3;                 // TMEM lane window of this warp
+    const int r = sp * 32 + lane;            // row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (wg ? C::TM_S1 : C::TM_S0);
+    const uint32_t tO = tmem + lane_off + (wg ? C::TM_O1 : C::TM_O0);
+    const uint32_t bar_s = bars + 8 * (C::B_S_FULL + wg), bar_p = bars + 8 * (C::B_P_FULL + wg);
+    const uint32_t bar_o = bars + 8 * (C::B_O_FULL + wg), bar_oe = bars + 8 * (C::B_O_EMPTY + wg);
+    uint32_t s_it = 0, o_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int bh, qp;
+      fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
+      const int qt = 2 * qp + wg;
+      const int nk = CAUSAL ? min(qt + 1, NKT) : NKT;
+      const int row = qt * C::BM + r;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < nk; ++j) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s, s_it & 1, FW_SM_S)))) break;
+        ++s_it;
+        tc_fence_after();
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        const int kbase = j * C::BN;
+        if ((CAUSAL && j == qt) || kbase + C::BN > N) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int key = kbase + c;
+            if (key >= N || (CAUSAL && key > row)) s[c] = -INFINITY;
+          }
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_ref, mx * scale_log2);
+        const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
+        const bool warp_rescale = __any_sync(0xffffffffu, need);
+        const float alpha = need ? ex2(m_ref - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
+        if (need) {
+          l *= alpha;
+          m_ref = m_new;
+        }
+        const float neg = -m_ref;
+        float lsum = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {  // 32 scores -> 16 packed bf16 pairs -> 16 TMEM columns
+          uint32_t p[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ex2(fmaf(s[32 * ch + 2 * c], scale_log2, neg));
+            const float p1 = ex2(fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg));
+            lsum += p0 + p1;
+            p[c] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + ch * 16, p);
+        }
+        // O holds PV of tiles 0..j-1 (the S MMA that signalled s_full was issued
+        // after them); rescale it before this tile's PV is issued.
+        if (warp_rescale && j > 0) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p);
+        l += lsum;
+      }
+      if (!ok) break;
+      // epilogue: O / l (bf16) and LSE (fp32, natural log of the scaled logits)
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_o, o_it & 1, FW_SM_O)))) break;
+      ++o_it;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = O + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_ld_wait();
+        reg_fence(o);
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+            w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+            w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+            w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+            dst[v] = w;
+          }
+        }
+      }
+      if (row < N) LSE[static_cast<size_t>(bh) * N + row] = (m_ref + __log2f(l)) * kLn2;
+      tc_fence_before();
+      mbar_arrive(bar_oe);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+}
+
+}  // namespace fa

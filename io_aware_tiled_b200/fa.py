@@ -1,0 +1,194 @@
+"""Thin Python binding of libfa.so (argument marshalling only).
+
+Every step of the attention path runs in the library's sm_100a kernels;
+torch supplies device memory and the current CUDA stream.  There is no CPU
+fallback: if the library is missing or the device is not an sm_100 GPU, the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+_HEADER = os.path.join(_build.INCLUDE, "fa.h")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = -1
+FA_ERR_ALIGNMENT = -2
+FA_ERR_UNSUPPORTED_DEVICE = -3
+FA_ERR_LAUNCH = -4
+FA_ERR_WORKSPACE = -5
+FA_ERR_TIMEOUT = -6
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(build_if_missing: bool = True):
+    """Load libfa.so (building it first if it is missing or older than its sources)."""
+    global _lib
+    if _lib is None:
+        if build_if_missing and _build.stale():
+            _build.build()
+        if not os.path.exists(_build.LIB):
+            raise RuntimeError(f"libfa.so is not built ({_build.LIB}); run io_aware_tiled_b200.build.build()")
+        lib = ctypes.CDLL(_build.LIB)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+        lib.fa_fwd.restype = i
+        lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        lib.fa_bwd_workspace_bytes.restype = sz
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+        lib.fa_bwd.restype = i
+        lib.fa_sync_status.argtypes = [vp]
+        lib.fa_sync_status.restype = i
+        lib.fa_last_error_word.argtypes = []
+        lib.fa_last_error_word.restype = ctypes.c_uint
+        lib.fa_status_string.argtypes = [i]
+        lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_bwd_set_phase_events.argtypes = [vp, vp, vp, vp]
+        lib.fa_bwd_set_phase_events.restype = None
+        lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+        lib.fa_selftest_wait_timeout.restype = i
+        _lib = lib
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/fa.h declares."""
+    text = open(_HEADER, encoding="utf-8").read()
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(fa_\w+)\s*\(", text, flags=re.M)
+
+
+def status_string(status: int) -> str:
+    return load_library().fa_status_string(int(status)).decode()
+
+
+def _stream_handle(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check_qkv(*ts: torch.Tensor):
+    t0 = ts[0]
+    if t0.dim() != 4:
+        raise ValueError("expected tensors of shape [B, H, N, d]")
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (no CPU path exists)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bfloat16")
+        if t.shape != t0.shape or t.device != t0.device:
+            raise ValueError("tensors must share shape and device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, N, d]")
+
+
+def _scale(scale, d):
+    return 0.0 if scale is None else float(scale)
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """O, LSE = attention(q, k, v); bf16 [B,H,N,d] in, (bf16 O, fp32 LSE [B,H,N]) out."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
+                        int(bool(causal)), _scale(scale, d), _stream_handle(q.device))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+    return o, l
+
+
+def workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
+             dq=None, dk=None, dv=None):
+    """dQ, dK, dV of sum(dO * O); inputs as produced by forward()."""
+    _check_qkv(q, k, v, o, do)
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous float32 [B, H, N]")
+    lib = load_library()
+    nbytes = int(lib.fa_bwd_workspace_bytes(B, H, N, d))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    with torch.cuda.device(q.device):
+        rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)),
+                        _scale(scale, d), ws.data_ptr(), ws.numel(), _stream_handle(q.device))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def sync_status(device=None) -> int:
+    """Synchronise the current stream and return the library's status code."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(load_library().fa_sync_status(_stream_handle(dev)))
+
+
+def set_backward_phase_events(events=None) -> None:
+    """Record four torch.cuda.Event objects around fa_bwd's kernels (D pass,
+    dK/dV, dQ); None stops.  The events must outlive their use."""
+    lib = load_library()
+    if events is None:
+        lib.fa_bwd_set_phase_events(None, None, None, None)
+    else:
+        lib.fa_bwd_set_phase_events(*[ctypes.c_void_p(e.cuda_event) for e in events])
+
+
+def last_error_word() -> int:
+    return int(load_library().fa_last_error_word())
+
+
+def selftest_wait_timeout(limit_us: int, device=None) -> int:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(load_library().fa_selftest_wait_timeout(int(limit_us), _stream_handle(dev)))
+
+
+class FlashAttentionFunction(torch.autograd.Function):
+    """autograd wrapper: forward and backward both run the library kernels."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal=False, scale=None):
+        o, lse = forward(q.contiguous(), k.contiguous(), v.contiguous(), causal, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.causal, ctx.scale = causal, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, o, do.contiguous(), lse, ctx.causal, ctx.scale)
+        return dq, dk, dv, None, None
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    return FlashAttentionFunction.apply(q, k, v, causal, scale)
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

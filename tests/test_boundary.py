@@ -1,0 +1,114 @@
+"""The C-ABI library loads, exports what include/fa.h declares, and rejects bad
+arguments before touching a GPU (these run on a machine without one)."""
+from __future__ import annotations
+
+import ctypes
+import re
+import subprocess
+
+import pytest
+import torch
+
+from io_aware_tiled_b200 import fa
+from io_aware_tiled_b200 import build as fa_build
+
+OK, EINVAL, EALIGN, EDEV, ELAUNCH, EWS, ETIMEOUT = 0, -1, -2, -3, -4, -5, -6
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return fa.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = fa.header_functions()
+    assert set(names) == {"fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_sync_status", "fa_last_error_word",
+                          "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events"}
+    out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (fa_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        getattr(lib, n)
+
+
+def test_status_strings(lib):
+    for code, name in [(OK, "FA_OK"), (EINVAL, "FA_ERR_INVALID_ARG"), (EALIGN, "FA_ERR_ALIGNMENT"),
+                       (EDEV, "FA_ERR_UNSUPPORTED_DEVICE"), (ELAUNCH, "FA_ERR_LAUNCH"),
+                       (EWS, "FA_ERR_WORKSPACE"), (ETIMEOUT, "FA_ERR_TIMEOUT")]:
+        assert fa.status_string(code) == name
+    assert fa.status_string(42) == "FA_ERR_UNKNOWN"
+
+
+def test_workspace_bytes(lib):
+    assert lib.fa_bwd_workspace_bytes(2, 16, 4096, 128) == 2 * 16 * 4096 * 4
+    assert lib.fa_bwd_workspace_bytes(8, 12, 1000, 64) == ((8 * 12 * 1000 * 4 + 255) // 256) * 256
+    assert lib.fa_bwd_workspace_bytes(1, 1, 0, 64) == 0
+    assert lib.fa_bwd_workspace_bytes(1, 1, 16, 96) == 0
+
+
+A = 1 << 20  # fake, 16-byte aligned, never dereferenced: validation stops before any device access
+
+
+def _fwd(lib, q=A, k=2 * A, v=3 * A, o=4 * A, lse=5 * A, B=1, H=1, N=128, d=64, causal=0, scale=0.0):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, None)
+
+
+def test_forward_rejects_bad_sizes(lib):
+    assert _fwd(lib, N=0) == EINVAL
+    assert _fwd(lib, N=-3) == EINVAL
+    assert _fwd(lib, B=0) == EINVAL
+    assert _fwd(lib, H=-1) == EINVAL
+    for d in (0, 32, 96, 256):
+        assert _fwd(lib, d=d) == EINVAL
+    assert _fwd(lib, B=2 ** 16, H=2 ** 16, N=2) == EINVAL  # B*H*N beyond 32-bit rows
+
+
+def test_forward_rejects_null_misaligned_and_overlap(lib):
+    assert _fwd(lib, q=0) == EINVAL
+    assert _fwd(lib, lse=0) == EINVAL
+    assert _fwd(lib, v=3 * A + 8) == EALIGN
+    assert _fwd(lib, o=4 * A + 2) == EALIGN
+    assert _fwd(lib, o=A) == EINVAL               # output aliases an input
+    assert _fwd(lib, lse=4 * A + 64) == EINVAL    # LSE inside O
+    assert _fwd(lib, scale=float("nan")) == EINVAL
+    assert _fwd(lib, scale=float("inf")) == EINVAL
+
+
+def test_forward_without_gpu_reports_unsupported_device(lib):
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _fwd(lib) == EDEV
+
+
+def _bwd(lib, ws=20 * A, ws_bytes=None, B=1, H=1, N=128, d=64, **ptrs):
+    p = dict(q=A, k=2 * A, v=3 * A, o=4 * A, do=5 * A, lse=6 * A, dq=7 * A, dk=8 * A, dv=9 * A)
+    p.update(ptrs)
+    nb = lib.fa_bwd_workspace_bytes(B, H, N, d) if ws_bytes is None else ws_bytes
+    return lib.fa_bwd(p["q"], p["k"], p["v"], p["o"], p["do"], p["lse"], p["dq"], p["dk"], p["dv"],
+                      B, H, N, d, 1, 0.0, ws, nb, None)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    assert _bwd(lib, N=0) == EINVAL
+    assert _bwd(lib, d=80) == EINVAL
+    assert _bwd(lib, do=0) == EINVAL
+    assert _bwd(lib, dk=8 * A + 4) == EALIGN
+    assert _bwd(lib, ws=0) == EWS
+    assert _bwd(lib, ws=20 * A + 8) == EWS
+    assert _bwd(lib, ws_bytes=16) == EWS
+    assert _bwd(lib, dq=A) == EINVAL              # dQ aliases Q
+    assert _bwd(lib, dv=8 * A) == EINVAL          # dV aliases dK
+    assert _bwd(lib, ws=9 * A) == EWS             # workspace aliases dV
+
+
+def test_selftest_rejects_bad_limit(lib):
+    assert lib.fa_selftest_wait_timeout(0, None) == EINVAL
+    assert lib.fa_selftest_wait_timeout(10_000_001, None) == EINVAL
+
+
+def test_python_binding_refuses_cpu_tensors():
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q)
+    with pytest.raises(ValueError):
+        fa.forward(q.float(), q.float(), q.float())

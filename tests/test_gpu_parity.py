@@ -1,0 +1,296 @@
+"""GPU parity: the sm_100a kernels (called through the C ABI) against the fp64 oracle.
+
+Every input is drawn by io_aware_tiled_b200.inputs (seeded, CPU, bf16); the
+oracle sees the same bf16 values widened to fp64.  Small shapes compare every
+element (several tiles plus a ragged tail); the five named workloads run at
+full size and compare whole heads or sampled rows the oracle computes one by
+one, plus properties that hold at any size.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_tiled_b200 import fa
+from io_aware_tiled_b200.configs import WORKLOADS
+from io_aware_tiled_b200.inputs import attention_inputs
+from tests.parity import check_grad, check_lse, check_o, f64, rel_frob, to_bf16_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda", 0)
+
+
+def _run_fwd(q, k, v, causal, scale=None):
+    dev = _dev()
+    o, lse = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal, scale)
+    assert fa.sync_status() == fa.FA_OK
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# forward, every element, shapes spanning several tiles and ragged tails
+# ---------------------------------------------------------------------------
+FWD_CASES = [
+    # B, H, N, d, causal, sigma_qk
+    (1, 1, 256, 64, False, 1.0),
+    (1, 1, 1, 64, False, 1.0),
+    (1, 1, 1, 128, True, 1.0),
+    (1, 2, 17, 64, True, 1.0),
+    (1, 1, 127, 128, False, 1.0),
+    (1, 1, 129, 128, True, 1.0),
+    (2, 2, 300, 128, False, 1.0),
+    (2, 2, 300, 128, True, 1.0),
+    (1, 2, 640, 64, True, 1.0),      # odd number of 128-row tiles
+    (1, 3, 1000, 64, True, 8.0),     # logits in the hundreds, ragged
+    (1, 3, 1000, 64, False, 8.0),
+    (1, 2, 777, 128, True, 2.0),
+    (1, 1, 2048, 128, False, 1.0),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,sigma", FWD_CASES)
+def test_forward_matches_oracle(B, H, N, d, causal, sigma):
+    q, k, v, _ = attention_inputs(B, H, N, d, seed=N + d, sigma_qk=sigma, with_do=False)
+    scale = 1.0 / d ** 0.5
+    o, lse = _run_fwd(q, k, v, causal)
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), causal, scale)
+    check_o(f64(o), ro, f"fwd {B,H,N,d,causal}")
+    check_lse(f64(lse), rl, f"fwd {B,H,N,d,causal}")
+
+
+def test_forward_explicit_scale_and_default():
+    q, k, v, _ = attention_inputs(1, 2, 200, 128, seed=5, with_do=False)
+    for scale in (0.05, 0.3):
+        o, lse = _run_fwd(q, k, v, True, scale)
+        ro, rl = oracle.forward(f64(q), f64(k), f64(v), True, scale)
+        check_o(f64(o), ro, f"scale {scale}")
+        check_lse(f64(lse), rl, f"scale {scale}")
+    o1, l1 = _run_fwd(q, k, v, False, None)
+    o2, l2 = _run_fwd(q, k, v, False, 1.0 / 128 ** 0.5)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------------------------
+# backward, every element
+# ---------------------------------------------------------------------------
+BWD_CASES = [
+    (1, 1, 256, 64, False, 1.0),
+    (1, 1, 1, 64, True, 1.0),
+    (1, 1, 129, 128, False, 1.0),
+    (1, 2, 300, 128, True, 1.0),
+    (2, 1, 640, 128, True, 1.0),
+    (1, 2, 1000, 64, False, 1.0),
+    (1, 2, 777, 64, True, 1.0),
+    (1, 1, 1024, 128, False, 1.0),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,sigma", BWD_CASES)
+def test_backward_matches_oracle(B, H, N, d, causal, sigma):
+    dev = _dev()
+    q, k, v, do = attention_inputs(B, H, N, d, seed=7 * N + d, sigma_qk=sigma)
+    scale = 1.0 / d ** 0.5
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = fa.forward(qd, kd, vd, causal)
+    dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, causal)
+    assert fa.sync_status() == fa.FA_OK
+    ref = oracle.backward(f64(q), f64(k), f64(v), f64(do), causal, scale)
+    what = f"bwd {B,H,N,d,causal}"
+    check_o(f64(o), ref["o"], what)
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check_grad(f64(g), ref[name], name, what)
+
+
+def test_backward_large_logits_against_both_forms_of_D():
+    """Logits in the hundreds: most rows are one-hot, so dQ and dK are tiny
+    differences.  Compare with the definitional oracle and, as a diagnostic
+    that isolates the bf16 format of O, with the oracle whose D uses its own O
+    rounded to bf16."""
+    dev = _dev()
+    B, H, N, d = 1, 2, 1000, 64
+    q, k, v, do = attention_inputs(B, H, N, d, seed=11, sigma_qk=8.0)
+    for causal in (False, True):
+        qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+        o, lse = fa.forward(qd, kd, vd, causal)
+        dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, causal)
+        assert fa.sync_status() == fa.FA_OK
+        ref = oracle.backward(f64(q), f64(k), f64(v), f64(do), causal, 1.0 / 8)
+        check_grad(f64(dv), ref["dv"], "dv", "sigma 8")
+        for name, g in (("dq", dq), ("dk", dk)):
+            check_grad(f64(g), ref[name], name, f"sigma 8 causal={causal}")
+
+
+# ---------------------------------------------------------------------------
+# the five named workloads at full size
+# ---------------------------------------------------------------------------
+def _sample_rows(rng, BH, N, n):
+    return np.sort(rng.choice(BH * N, size=min(n, BH * N), replace=False))
+
+
+def _full_forward_check(w, causal, heads_full, n_random_rows):
+    dev = _dev()
+    q, k, v, do = attention_inputs(w.B, w.H, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk, with_do=w.backward)
+    o, lse = _run_fwd(q, k, v, causal)
+    o_np, lse_np = f64(o).reshape(-1, w.d), f64(lse).reshape(-1)
+    rng = np.random.default_rng(0)
+    rows = [np.arange(h * w.N, (h + 1) * w.N) for h in heads_full]
+    rows.append(_sample_rows(rng, w.B * w.H, w.N, n_random_rows))
+    rows = np.unique(np.concatenate(rows))
+    ro, rl = oracle.forward_rows(f64(q), f64(k), f64(v), causal, w.scale, rows)
+    check_o(o_np[rows], ro, f"{w.name} causal={causal}")
+    check_lse(lse_np[rows], rl, f"{w.name} causal={causal}")
+    # properties at every row: finite; causal row 0 of every head is exactly V[0]
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    if causal:
+        assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0])
+    return q, k, v, do, o, lse
+
+
+def _full_backward_check(w, causal, q, k, v, do, o, lse, heads, n_rows):
+    dev = _dev()
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, causal)
+    assert fa.sync_status() == fa.FA_OK
+    rng = np.random.default_rng(1)
+    dq_np, dk_np, dv_np = (f64(t).reshape(w.B * w.H, w.N, w.d) for t in (dq, dk, dv))
+    for bh in heads:
+        qr = np.sort(rng.choice(w.N, size=min(n_rows, w.N), replace=False))
+        kr = np.sort(rng.choice(w.N, size=min(n_rows, w.N), replace=False))
+        qr[0], kr[0] = 0, w.N - 1
+        ref = oracle.backward_sampled(f64(q), f64(k), f64(v), f64(do), causal, w.scale, bh, qr, kr)
+        what = f"{w.name} causal={causal} head {bh}"
+        check_grad(dq_np[bh][qr], ref["dq"], "dq", what)
+        check_grad(dk_np[bh][kr], ref["dk"], "dk", what)
+        check_grad(dv_np[bh][kr], ref["dv"], "dv", what)
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+
+
+def test_workload_pr1_full():
+    w = WORKLOADS["pr1_b1h1n256d64"]
+    q, k, v, _ = attention_inputs(w.B, w.H, w.N, w.d, seed=w.seed, with_do=False)
+    o, lse = _run_fwd(q, k, v, False)
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), False, w.scale)
+    check_o(f64(o), ro, w.name)
+    check_lse(f64(lse), rl, w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_workload_fwd_b2h16n4096d128(causal):
+    w = WORKLOADS["fwd_b2h16n4096d128"]
+    _full_forward_check(w, causal, heads_full=[0, 31], n_random_rows=512)
+
+
+def test_workload_train_b4h32n2048d128():
+    w = WORKLOADS["train_b4h32n2048d128"]
+    q, k, v, do, o, lse = _full_forward_check(w, True, heads_full=[0, 127], n_random_rows=512)
+    _full_backward_check(w, True, q, k, v, do, o, lse, heads=[0, 77, 127], n_rows=64)
+
+
+def test_workload_long_b1h16n16384d128():
+    w = WORKLOADS["long_b1h16n16384d128"]
+    q, k, v, do, o, lse = _full_forward_check(w, True, heads_full=[], n_random_rows=384)
+    _full_backward_check(w, True, q, k, v, do, o, lse, heads=[15], n_rows=48)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_workload_ragged_b8h12n1000d64(causal):
+    w = WORKLOADS["ragged_b8h12n1000d64"]
+    q, k, v, do, o, lse = _full_forward_check(w, causal, heads_full=[0, 50, 95], n_random_rows=1024)
+    _full_backward_check(w, causal, q, k, v, do, o, lse, heads=[0, 95], n_rows=64)
+
+
+# ---------------------------------------------------------------------------
+# edge cases, guard bands, determinism, autograd wrapper, errors, fault detection
+# ---------------------------------------------------------------------------
+def test_outputs_stay_inside_their_buffers():
+    """Canary guard bands before and after O and LSE are untouched."""
+    dev = _dev()
+    B, H, N, d = 1, 3, 333, 128
+    q, k, v, _ = attention_inputs(B, H, N, d, seed=3, with_do=False)
+    guard = 4096
+    n_o, n_l = B * H * N * d, B * H * N
+    obuf = torch.full((n_o + 2 * guard,), -7.0, dtype=torch.bfloat16, device=dev)
+    lbuf = torch.full((n_l + 2 * guard,), 123.25, dtype=torch.float32, device=dev)
+    o = obuf[guard:guard + n_o].view(B, H, N, d)
+    l = lbuf[guard:guard + n_l].view(B, H, N)
+    fa.forward(q.to(dev), k.to(dev), v.to(dev), True, out=o, lse=l)
+    assert fa.sync_status() == fa.FA_OK
+    assert (obuf[:guard] == -7.0).all() and (obuf[guard + n_o:] == -7.0).all()
+    assert (lbuf[:guard] == 123.25).all() and (lbuf[guard + n_l:] == 123.25).all()
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), True, 1 / d ** 0.5)
+    check_o(f64(o), ro, "guarded")
+
+
+def test_gradient_outputs_stay_inside_their_buffers():
+    dev = _dev()
+    B, H, N, d = 1, 2, 200, 64
+    q, k, v, do = attention_inputs(B, H, N, d, seed=4)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = fa.forward(qd, kd, vd, False)
+    guard, n = 2048, B * H * N * d
+    bufs = [torch.full((n + 2 * guard,), 3.5, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    views = [b[guard:guard + n].view(B, H, N, d) for b in bufs]
+    fa.backward(qd, kd, vd, o, dod, lse, False, dq=views[0], dk=views[1], dv=views[2])
+    assert fa.sync_status() == fa.FA_OK
+    for b in bufs:
+        assert (b[:guard] == 3.5).all() and (b[guard + n:] == 3.5).all()
+
+
+def test_forward_and_backward_are_deterministic():
+    dev = _dev()
+    q, k, v, do = attention_inputs(1, 4, 1000, 128, seed=9)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    for causal in (False, True):
+        o1, l1 = fa.forward(qd, kd, vd, causal)
+        o2, l2 = fa.forward(qd, kd, vd, causal)
+        g1 = fa.backward(qd, kd, vd, o1, dod, l1, causal)
+        g2 = fa.backward(qd, kd, vd, o1, dod, l1, causal)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        for a, b in zip(g1, g2):
+            assert torch.equal(a, b)
+
+
+def test_autograd_wrapper_runs_library_kernels():
+    dev = _dev()
+    q, k, v, do = attention_inputs(1, 2, 256, 64, seed=12)
+    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
+    o = fa.attention(qd, kd, vd, True)
+    o.backward(do.to(dev))
+    o2, lse = fa.forward(qd.detach(), kd.detach(), vd.detach(), True)
+    g = fa.backward(qd.detach(), kd.detach(), vd.detach(), o2, do.to(dev), lse, True)
+    assert torch.equal(o.detach(), o2)
+    for t, ref in zip((qd, kd, vd), g):
+        assert torch.equal(t.grad, ref)
+
+
+def test_invalid_arguments_on_gpu():
+    dev = _dev()
+    q = torch.zeros(1, 1, 64, 96, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(fa.FaError) as e:
+        fa.forward(q, q.clone(), q.clone())
+    assert e.value.status == fa.FA_ERR_INVALID_ARG
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(ValueError):
+        fa.forward(q, q.float(), q)
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    """A wait on a barrier nothing signals runs out after 2 ms; the library
+    reports FA_ERR_TIMEOUT and the next launches work normally."""
+    dev = _dev()
+    assert fa.selftest_wait_timeout(2000) == fa.FA_OK
+    assert fa.sync_status() == fa.FA_ERR_TIMEOUT
+    assert fa.last_error_word() == (255 << 8) | 1
+    assert fa.sync_status() == fa.FA_OK  # cleared
+    q, k, v, _ = attention_inputs(1, 1, 256, 64, seed=0, with_do=False)
+    o, lse = _run_fwd(q, k, v, False)
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), False, 1 / 8)
+    check_o(f64(o), ro, "after timeout")

@@ -346,3 +346,13 @@ def test_input_recipe_is_seeded_and_bf16():
     assert 5.0 < float(a[0].float().std()) < 11.0 and 0.7 < float(a[2].float().std()) < 1.3
     with pytest.raises(ValueError):
         attention_inputs(1, 1, 0, 64)
+
+
+def test_parity_helpers_format_floor():
+    """The O check's format floor: half a bf16 spacing, e.g. 1/128 on [2, 4)."""
+    from tests.parity import half_ulp_bf16, o_excess_error
+    np.testing.assert_array_equal(half_ulp_bf16([1.0, 1.5, 2.0, 3.9, 0.25]),
+                                  [2 ** -8, 2 ** -8, 2 ** -7, 2 ** -7, 2 ** -10])
+    # a one-spacing flip next to a midpoint is within the budget, an error of 0.02 is not
+    assert o_excess_error([3.0 + 2 ** -6], [3.0 + 2 ** -7 + 1e-6]) < 1e-2
+    assert o_excess_error([3.02], [3.0]) > 1e-2
