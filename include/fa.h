@@ -98,6 +98,13 @@ int fa_sync_status(void* stream);
 unsigned int fa_last_error_word(void);
 
 /*
+ * The cause of the last FA_ERR_LAUNCH returned by this library, for
+ * diagnosis: a cudaError_t value, or 100000 + the CUresult of a failed
+ * tensor-map encode (0 if none).
+ */
+int fa_last_cuda_error(void);
+
+/*
  * Optional per-kernel timing of fa_bwd (profiling aid).  When set, fa_bwd
  * records the four cudaEvent_t handles (passed as void*) on its stream:
  * e0 before the D pass, e1 before the dK/dV kernel, e2 before the dQ

@@ -29,16 +29,23 @@ EncodeTiledFn encode_fn() {
 
 // 3-D view [BH][N][d] of a bf16 [B,H,N,d] tensor; box = 64 columns x box_rows
 // rows x 1 head, 128-byte swizzle.  Rows past N read as zero within the head.
+int g_last_encode_error = 0;  // CUresult of the last failed tensor-map encode (diagnosis)
+
 bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    g_last_encode_error = -1;
+    return false;
+  }
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_encode_error = static_cast<int>(r);
+  return r == CUDA_SUCCESS;
 }
 
 constexpr int kMaxDevices = 64;
@@ -91,6 +98,26 @@ int device_ready(int* sms) {
 }
 
 cudaEvent_t g_phase_events[4] = {nullptr, nullptr, nullptr, nullptr};
+int g_last_cuda_error = 0;
+
+// Status of the launches just made.  Errors left pending by earlier, unrelated
+// runtime calls on this thread are cleared before launching (see
+// clear_stale_error), so an error seen here belongs to these launches.
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return FA_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_LAUNCH;
+}
+void clear_stale_error() { (void)cudaGetLastError(); }
+
+// A tensor-map encode failed: reported as FA_ERR_LAUNCH with
+// fa_last_cuda_error() = 100000 + the driver's CUresult (or 99999 if the
+// driver entry point could not be found).
+int encode_failed() {
+  g_last_cuda_error = 100000 + g_last_encode_error;
+  return FA_ERR_LAUNCH;
+}
 std::mutex g_events_mu;
 
 bool is_device_ptr(const void* p) {
@@ -164,7 +191,8 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, BH, N, d, 128) || !make_map(&mk, K, BH, N, d, 128) || !make_map(&mv, V, BH, N, d, 128))
-    return FA_ERR_LAUNCH;
+    return encode_failed();
+  clear_stale_error();
   const int nqt = (N + 127) / 128, units = BH * ((nqt + 1) / 2);
   const int grid = units < sms ? units : sms;
   const float sl2 = sc * fa::kLog2e;
@@ -177,7 +205,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
     if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
     else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
   }
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return launch_status();
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -225,8 +253,9 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
       !make_map(&mk128, K, BH, N, d, 128) || !make_map(&mv128, V, BH, N, d, 128) ||
       !make_map(&mq128, Q, BH, N, d, 128) || !make_map(&mdo128, dO, BH, N, d, 128) ||
       !make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64))
-    return FA_ERR_LAUNCH;
+    return encode_failed();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  clear_stale_error();
   float* Dvec = static_cast<float*>(workspace);
   const long long rows = static_cast<long long>(BH) * N;
   const float sl2 = sc * fa::kLog2e;
@@ -278,7 +307,7 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
       mark(3);
     }
   }
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return launch_status();
 }
 
 static unsigned int g_last_error_word = 0;
@@ -307,6 +336,8 @@ int fa_sync_status(void* stream) {
 
 unsigned int fa_last_error_word(void) { return g_last_error_word; }
 
+int fa_last_cuda_error(void) { return g_last_cuda_error; }
+
 }  // extern "C"
 
 namespace fa {
@@ -329,7 +360,8 @@ extern "C" int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   int sms = 0;
   int rc = device_ready(&sms);
   if (rc) return rc;
+  clear_stale_error();
   fa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<unsigned long long>(limit_us) * 1000ull);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  return launch_status();
 }

@@ -30,7 +30,10 @@ FA_ERR_TIMEOUT = -6
 class FaError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} ({status})")
+        extra = ""
+        if status == FA_ERR_LAUNCH:
+            extra = f", cudaError {load_library().fa_last_cuda_error()}"
+        super().__init__(f"{what}: {status_string(status)} ({status}{extra})")
 
 
 _lib = None
@@ -60,6 +63,8 @@ def load_library(build_if_missing: bool = True):
         lib.fa_sync_status.restype = i
         lib.fa_last_error_word.argtypes = []
         lib.fa_last_error_word.restype = ctypes.c_uint
+        lib.fa_last_cuda_error.argtypes = []
+        lib.fa_last_cuda_error.restype = i
         lib.fa_status_string.argtypes = [i]
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_bwd_set_phase_events.argtypes = [vp, vp, vp, vp]
@@ -157,6 +162,9 @@ def set_backward_phase_events(events=None) -> None:
     if events is None:
         lib.fa_bwd_set_phase_events(None, None, None, None)
     else:
+        for e in events:  # torch creates the CUDA event on its first record
+            if e.cuda_event == 0:
+                e.record()
         lib.fa_bwd_set_phase_events(*[ctypes.c_void_p(e.cuda_event) for e in events])
 
 
