@@ -50,7 +50,8 @@ typedef enum {
   FA_ERR_UNSUPPORTED_DEVICE = -3, /* current device is not sm_100, or a pointer is not device memory */
   FA_ERR_LAUNCH = -4,             /* a CUDA call or kernel launch failed */
   FA_ERR_WORKSPACE = -5,          /* backward workspace missing, misaligned or too small */
-  FA_ERR_TIMEOUT = -6             /* a kernel's internal wait ran out (reported by fa_sync_status) */
+  FA_ERR_TIMEOUT = -6,            /* a kernel's internal wait ran out (reported by fa_sync_status) */
+  FA_ERR_TOO_LARGE = -7           /* fa_bwd_noalloc: B*H*N exceeds FA_NOALLOC_MAX_ROWS */
 } fa_status;
 
 /*
@@ -83,6 +84,31 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
            void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd for callers that cannot allocate device memory -- for example a
+ * plugin whose host runtime hands it only its input and output buffers, or
+ * code running under a memory pool that must not grow.  The paper has no
+ * counterpart to this entry point.
+ *
+ * Same arguments, semantics and outputs as fa_bwd, minus the workspace: the
+ * D = rowsum(dO * O) vector lives in a fixed array inside the library
+ * (FA_NOALLOC_MAX_ROWS fp32 entries = 4 MiB, held on every GPU that loads the
+ * library until the process exits).  The call itself allocates nothing.
+ *  - Sizes: B*H*N must not exceed FA_NOALLOC_MAX_ROWS, else FA_ERR_TOO_LARGE
+ *    (nothing is launched).
+ *  - Set-up: the first call on each device looks up the array's device address
+ *    (with that device current); make that first call before any stream
+ *    capture.
+ *  - The array is shared by every call on a device and keeps the last call's
+ *    contents; each call overwrites the part it uses before reading it.  Calls
+ *    that overlap on the GPU (different streams, no ordering between them) race
+ *    on the array: order them or use fa_bwd with separate workspaces.
+ */
+#define FA_NOALLOC_MAX_ROWS (1 << 20)
+int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                   void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
+                   void* stream);
 
 /*
  * Synchronises `stream`, then reports: FA_ERR_LAUNCH if a CUDA error is

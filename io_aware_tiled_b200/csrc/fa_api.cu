@@ -164,6 +164,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_TOO_LARGE: return "FA_ERR_TOO_LARGE";
     default: return "FA_ERR_UNKNOWN";
   }
 }
@@ -364,4 +365,49 @@ extern "C" int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   fa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<unsigned long long>(limit_us) * 1000ull);
   return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// fa_bwd_noalloc: the backward with its D vector in a fixed device array, for
+// callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+namespace {
+// FA_NOALLOC_MAX_ROWS fp32 entries; every device that loads the library holds
+// it until the process exits.  In host code this name is only a stand-in:
+// kernels get the device address from cudaGetSymbolAddress below.
+__device__ __align__(256) float g_noalloc_d[FA_NOALLOC_MAX_ROWS];
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                              const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                              int causal, float scale, void* stream) {
+  int rc = check_sizes(B, H, N, d);
+  if (rc) return rc;
+  if (static_cast<long long>(B) * H * N > FA_NOALLOC_MAX_ROWS) return FA_ERR_TOO_LARGE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_UNSUPPORTED_DEVICE;
+  }
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {  // set-up, once per device, with that device current
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_d);
+      if (e != cudaSuccess || !p) {
+        g_last_cuda_error = static_cast<int>(e);
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+      }
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  // D is written in full by the first kernel before anything reads it, so the
+  // array needs no clearing between calls.
+  return fa_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, scratch,
+                static_cast<size_t>(FA_NOALLOC_MAX_ROWS) * sizeof(float), stream);
 }

@@ -25,6 +25,8 @@ FA_ERR_UNSUPPORTED_DEVICE = -3
 FA_ERR_LAUNCH = -4
 FA_ERR_WORKSPACE = -5
 FA_ERR_TIMEOUT = -6
+FA_ERR_TOO_LARGE = -7
+NOALLOC_MAX_ROWS = 1 << 20
 
 
 class FaError(RuntimeError):
@@ -59,6 +61,8 @@ def load_library(build_if_missing: bool = True):
         lib.fa_bwd_workspace_bytes.restype = sz
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
         lib.fa_bwd.restype = i
+        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+        lib.fa_bwd_noalloc.restype = i
         lib.fa_sync_status.argtypes = [vp]
         lib.fa_sync_status.restype = i
         lib.fa_last_error_word.argtypes = []
@@ -146,6 +150,29 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
                         _scale(scale, d), ws.data_ptr(), ws.numel(), _stream_handle(q.device))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def backward_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, dq=None, dk=None,
+                     dv=None):
+    """backward() without a workspace: the library's fixed 4 MiB device array
+    holds D (B*H*N <= NOALLOC_MAX_ROWS).  For callers that cannot allocate
+    device memory; pass preallocated dq/dk/dv to allocate nothing at all.
+    Calls that overlap on the GPU share the array and race."""
+    _check_qkv(q, k, v, o, do)
+    B, H, N, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous float32 [B, H, N]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        rc = lib.fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                                int(bool(causal)), _scale(scale, d), _stream_handle(q.device))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

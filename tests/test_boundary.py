@@ -24,7 +24,7 @@ def test_every_declared_symbol_is_exported(lib):
     names = fa.header_functions()
     assert set(names) == {"fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_sync_status", "fa_last_error_word",
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
-                          "fa_last_cuda_error"}
+                          "fa_last_cuda_error", "fa_bwd_noalloc"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:
@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_status_strings(lib):
     for code, name in [(OK, "FA_OK"), (EINVAL, "FA_ERR_INVALID_ARG"), (EALIGN, "FA_ERR_ALIGNMENT"),
                        (EDEV, "FA_ERR_UNSUPPORTED_DEVICE"), (ELAUNCH, "FA_ERR_LAUNCH"),
-                       (EWS, "FA_ERR_WORKSPACE"), (ETIMEOUT, "FA_ERR_TIMEOUT")]:
+                       (EWS, "FA_ERR_WORKSPACE"), (ETIMEOUT, "FA_ERR_TIMEOUT"), (-7, "FA_ERR_TOO_LARGE")]:
         assert fa.status_string(code) == name
     assert fa.status_string(42) == "FA_ERR_UNKNOWN"
 
