@@ -68,6 +68,13 @@ int device_ready(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_UNSUPPORTED_DEVICE;
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED_DEVICE;
+  // Binds the device's primary context to this thread (a thread that only had
+  // its device set, e.g. an autograd worker, may have none yet); the tensor-map
+  // encoder is a driver call and needs it.
+  if (cudaSetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_UNSUPPORTED_DEVICE;
+  }
   std::lock_guard<std::mutex> lock(g_dev_mu);
   DeviceInfo& di = g_dev[dev];
   if (di.checked == 0) {

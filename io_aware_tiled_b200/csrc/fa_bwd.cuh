@@ -179,43 +179,43 @@ __global__ void __launch_bounds__(DkdvCfg<D>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // whole warp, warp-uniform values; one elected lane issues each MMA / commit
       constexpr uint32_t IDESC_T = idesc_bf16(128, C::BQ, false, false);  // S^T, dP^T: M=128 keys, N=64 queries
       constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);        // dV, dK: B operand MN-major
       auto issue_t = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(d_tmem, sdesc_sw128(a_smem + (kk >> 2) * C::KCHUNK + (kk & 3) * 32, 16, 1024),
+          mma_ss_warp(d_tmem, sdesc_sw128(a_smem + (kk >> 2) * C::KCHUNK + (kk & 3) * 32, 16, 1024),
                  sdesc_sw128(b_smem + (kk >> 2) * C::QCHUNK + (kk & 3) * 32, 16, 1024), IDESC_T,
                  kk > 0 ? 1u : 0u);
       };
       auto issue_g = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 16 * 128, C::QCHUNK, 1024), IDESC_G,
+          mma_ts_warp(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 16 * 128, C::QCHUNK, 1024), IDESC_G,
                  (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bars + 8 * C::B_KV_FULL, 0, BW_MMA_KV);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_KV_FULL, 0, BW_MMA_KV));
       tc_fence_after();
       for (int it = 0; it <= nt && ok; ++it) {
         if (it < nt) {
           const int st = it % C::ST, b = it & 1;
-          if (!(ok = mbar_wait(bars + 8 * (C::B_Q_FULL + st), (it / C::ST) & 1, BW_MMA_Q))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_FULL + st), (it / C::ST) & 1, BW_MMA_Q)))) break;
           tc_fence_after();
           issue_t(tmem + C::TM_S + b * 64, sK, sQ + st * C::Q_TILE);
           issue_t(tmem + C::TM_DP + b * 64, sV, sdO + st * C::Q_TILE);
-          tc_commit(bars + 8 * (C::B_S_FULL + b));
+          tc_commit_warp(bars + 8 * (C::B_S_FULL + b));
         }
         if (it > 0) {
           const int pit = it - 1, pst = pit % C::ST, pb = pit & 1;
-          if (!(ok = mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BW_MMA_P))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BW_MMA_P)))) break;
           tc_fence_after();
           issue_g(tmem + C::TM_DV, tmem + C::TM_S + pb * 64, sdO + pst * C::Q_TILE, pit > 0);
           issue_g(tmem + C::TM_DK, tmem + C::TM_DP + pb * 64, sQ + pst * C::Q_TILE, pit > 0);
-          tc_commit(bars + 8 * (C::B_Q_EMPTY + pst));
+          tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + pst));
         }
       }
-      if (ok) tc_commit(bars + 8 * C::B_DKV_FULL);
+      if (ok) tc_commit_warp(bars + 8 * C::B_DKV_FULL);
     }
   } else {
     // ------------------------------------------------------------ softmax-gradient warpgroup
@@ -404,40 +404,40 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // whole warp, warp-uniform values; one elected lane issues each MMA / commit
       constexpr uint32_t IDESC_S = idesc_bf16(128, C::BK, false, false);  // S, dP: M=128 queries, N=64 keys
       constexpr uint32_t IDESC_Q = idesc_bf16(128, D, false, true);       // dQ: B (K tile) MN-major
       auto issue_s = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(d_tmem, sdesc_sw128(a_smem + (kk >> 2) * C::QCHUNK + (kk & 3) * 32, 16, 1024),
+          mma_ss_warp(d_tmem, sdesc_sw128(a_smem + (kk >> 2) * C::QCHUNK + (kk & 3) * 32, 16, 1024),
                  sdesc_sw128(b_smem + (kk >> 2) * C::KCHUNK + (kk & 3) * 32, 16, 1024), IDESC_S,
                  kk > 0 ? 1u : 0u);
       };
-      bool ok = mbar_wait(bars + 8 * C::B_Q_FULL, 0, BQ_MMA_Q);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_FULL, 0, BQ_MMA_Q));
       tc_fence_after();
       for (int it = 0; it <= nt && ok; ++it) {
         if (it < nt) {
           const int st = it % C::ST, b = it & 1;
-          if (!(ok = mbar_wait(bars + 8 * (C::B_KV_FULL + st), (it / C::ST) & 1, BQ_MMA_KV))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_KV_FULL + st), (it / C::ST) & 1, BQ_MMA_KV)))) break;
           tc_fence_after();
           issue_s(tmem + C::TM_S + b * 64, sQ, sK + st * C::K_TILE);
           issue_s(tmem + C::TM_DP + b * 64, sdO, sV + st * C::K_TILE);
-          tc_commit(bars + 8 * (C::B_S_FULL + b));
+          tc_commit_warp(bars + 8 * (C::B_S_FULL + b));
         }
         if (it > 0) {
           const int pit = it - 1, pst = pit % C::ST, pb = pit & 1;
-          if (!(ok = mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BQ_MMA_P))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BQ_MMA_P)))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk)
-            mma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + pb * 64 + kk * 8,
+            mma_ts_warp(tmem + C::TM_DQ, tmem + C::TM_DP + pb * 64 + kk * 8,
                    sdesc_sw128(sK + pst * C::K_TILE + kk * 16 * 128, C::KCHUNK, 1024), IDESC_Q,
                    (pit > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bars + 8 * (C::B_KV_EMPTY + pst));
+          tc_commit_warp(bars + 8 * (C::B_KV_EMPTY + pst));
         }
       }
-      if (ok) tc_commit(bars + 8 * C::B_DQ_FULL);
+      if (ok) tc_commit_warp(bars + 8 * C::B_DQ_FULL);
     }
   } else {
     const int sp = warp & 3;

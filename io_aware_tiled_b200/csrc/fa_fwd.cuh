@@ -72,10 +72,18 @@ enum FwdWaitSite : unsigned int {
   FW_PROD_Q = 1, FW_PROD_K, FW_PROD_V, FW_MMA_Q, FW_MMA_K, FW_MMA_V, FW_MMA_P, FW_MMA_OE, FW_SM_S, FW_SM_O
 };
 
+// Unit order.  Non-causal: head-major, so the CTAs running at the same time
+// share a few heads' K and V in L2.  Causal: longest units (last query pairs)
+// first across all heads, so the persistent CTAs finish together.
 __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool causal, int& bh, int& qp) {
-  const int r = u / BH;
-  bh = u - r * BH;
-  qp = causal ? (NP - 1 - r) : r;  // causal: longest units first
+  if (causal) {
+    const int r = u / BH;
+    bh = u - r * BH;
+    qp = NP - 1 - r;
+  } else {
+    bh = u / NP;
+    qp = u - bh * NP;
+  }
 }
 
 template <int D, bool CAUSAL>
@@ -167,7 +175,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
     } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop with warp-uniform values; one elected lane
+    // issues each tcgen05.mma / commit.
+    {
       constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
       // S = Q_t K_j^T: D/16 steps of K = 16 (32 bytes inside a 128-byte row; the
@@ -177,7 +187,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll 1
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(d_tmem, sdesc_make(sdesc_lo(a_smem + off, 16), hi), sdesc_make(sdesc_lo(b_smem + off, 16), hi),
+          mma_ss_warp(d_tmem, sdesc_make(sdesc_lo(a_smem + off, 16), hi), sdesc_make(sdesc_lo(b_smem + off, 16), hi),
                  IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
@@ -187,7 +197,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const uint32_t hi = sdesc_hi(1024);
 #pragma unroll 1
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts(d_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_smem + kk * 16 * 128, C::CHUNK), hi), IDESC_PV,
+          mma_ts_warp(d_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_smem + kk * 16 * 128, C::CHUNK), hi), IDESC_PV,
                  (acc || kk > 0) ? 1u : 0u);
       };
       uint32_t kv_it = 0, q_it = 0, unit_it = 0;
@@ -198,63 +208,63 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         (void)bh;
         const int nk0 = CAUSAL ? min(2 * qp + 1, NKT) : NKT;
         const int nk1 = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
-        bool ok = mbar_wait(bars + 8 * C::B_Q_FULL, q_it & 1, FW_MMA_Q);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_FULL, q_it & 1, FW_MMA_Q));
         ++q_it;
         if (!ok) break;
         tc_fence_after();
         {
           const int s = kv_it % C::ST;
-          if (!mbar_wait(bars + 8 * (C::B_K_FULL + s), (kv_it / C::ST) & 1, FW_MMA_K)) break;
+          if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_K_FULL + s), (kv_it / C::ST) & 1, FW_MMA_K))) break;
           tc_fence_after();
           issue_s(tmem + C::TM_S0, sQ, sK + s * C::KV_TILE);
-          tc_commit(bars + 8 * (C::B_S_FULL + 0));
+          tc_commit_warp(bars + 8 * (C::B_S_FULL + 0));
           issue_s(tmem + C::TM_S1, sQ + C::Q_TILE, sK + s * C::KV_TILE);
-          tc_commit(bars + 8 * (C::B_S_FULL + 1));
-          tc_commit(bars + 8 * (C::B_K_EMPTY + s));
+          tc_commit_warp(bars + 8 * (C::B_S_FULL + 1));
+          tc_commit_warp(bars + 8 * (C::B_K_EMPTY + s));
         }
         for (int j = 0; j < nk1 && ok; ++j) {
           const uint32_t it = kv_it + j;
           const int s = it % C::ST;
-          if (!(ok = mbar_wait(bars + 8 * (C::B_V_FULL + s), (it / C::ST) & 1, FW_MMA_V))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_V_FULL + s), (it / C::ST) & 1, FW_MMA_V)))) break;
           tc_fence_after();
           if (j < nk0) {
-            if (!(ok = mbar_wait(bars + 8 * (C::B_P_FULL + 0), p_ph0, FW_MMA_P))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + 0), p_ph0, FW_MMA_P)))) break;
             p_ph0 ^= 1;
-            if (j == 0 && !(ok = mbar_wait(bars + 8 * (C::B_O_EMPTY + 0), (unit_it & 1) ^ 1, FW_MMA_OE))) break;
+            if (j == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_O_EMPTY + 0), (unit_it & 1) ^ 1, FW_MMA_OE)))) break;
             tc_fence_after();
             issue_pv(tmem + C::TM_O0, tmem + C::TM_S0, sV + s * C::KV_TILE, j > 0);
-            if (j == nk0 - 1) tc_commit(bars + 8 * (C::B_O_FULL + 0));
+            if (j == nk0 - 1) tc_commit_warp(bars + 8 * (C::B_O_FULL + 0));
           }
           const bool more = j + 1 < nk1;
           const int sn = (it + 1) % C::ST;
           if (more) {
-            if (!(ok = mbar_wait(bars + 8 * (C::B_K_FULL + sn), ((it + 1) / C::ST) & 1, FW_MMA_K))) break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_K_FULL + sn), ((it + 1) / C::ST) & 1, FW_MMA_K)))) break;
             tc_fence_after();
             if (j + 1 < nk0) {
               issue_s(tmem + C::TM_S0, sQ, sK + sn * C::KV_TILE);
-              tc_commit(bars + 8 * (C::B_S_FULL + 0));
+              tc_commit_warp(bars + 8 * (C::B_S_FULL + 0));
             }
           }
-          if (!(ok = mbar_wait(bars + 8 * (C::B_P_FULL + 1), p_ph1, FW_MMA_P))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + 1), p_ph1, FW_MMA_P)))) break;
           p_ph1 ^= 1;
-          if (j == 0 && !(ok = mbar_wait(bars + 8 * (C::B_O_EMPTY + 1), (unit_it & 1) ^ 1, FW_MMA_OE))) break;
+          if (j == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_O_EMPTY + 1), (unit_it & 1) ^ 1, FW_MMA_OE)))) break;
           tc_fence_after();
           issue_pv(tmem + C::TM_O1, tmem + C::TM_S1, sV + s * C::KV_TILE, j > 0);
-          tc_commit(bars + 8 * (C::B_V_EMPTY + s));
-          if (j == nk1 - 1) tc_commit(bars + 8 * (C::B_O_FULL + 1));
+          tc_commit_warp(bars + 8 * (C::B_V_EMPTY + s));
+          if (j == nk1 - 1) tc_commit_warp(bars + 8 * (C::B_O_FULL + 1));
           if (more) {
             issue_s(tmem + C::TM_S1, sQ + C::Q_TILE, sK + sn * C::KV_TILE);
-            tc_commit(bars + 8 * (C::B_S_FULL + 1));
-            tc_commit(bars + 8 * (C::B_K_EMPTY + sn));
+            tc_commit_warp(bars + 8 * (C::B_S_FULL + 1));
+            tc_commit_warp(bars + 8 * (C::B_K_EMPTY + sn));
           }
         }
         if (!ok) break;
-        tc_commit(bars + 8 * C::B_Q_EMPTY);
+        tc_commit_warp(bars + 8 * C::B_Q_EMPTY);
         kv_it += nk1;
       }
       // The last unit's Q_EMPTY arrival is the last one this thread's commits
       // make; wait for it so no arrival lands after the CTA has exited.
-      if (q_it > 0) mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it - 1) & 1, FW_MMA_Q);
+      if (q_it > 0) (void)__all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it - 1) & 1, FW_MMA_Q));
     }
     }
     // teardown (each branch has its own, so the register regions never merge)
@@ -305,9 +315,19 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (key >= N || (CAUSAL && key > row)) s[c] = -INFINITY;
           }
         }
-        float mx = s[0];
+        // row max: 8 independent partial maxima, then a tree (short dependency chains)
+        float pm[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) pm[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
+        const float mx = pm[0];
         const float m_new = fmaxf(m_ref, mx * scale_log2);
         const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
         const bool warp_rescale = __any_sync(0xffffffffu, need);
@@ -317,7 +337,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           m_ref = m_new;
         }
         const float neg = -m_ref;
-        float lsum = 0.f;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 32 scores -> 16 packed bf16 pairs -> 16 TMEM columns
           uint32_t p[16];
@@ -325,11 +345,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int c = 0; c < 16; ++c) {
             const float p0 = ex2(fmaf(s[32 * ch + 2 * c], scale_log2, neg));
             const float p1 = ex2(fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg));
-            lsum += p0 + p1;
+            ps[c & 7] += p0 + p1;
             p[c] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + ch * 16, p);
         }
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) ps[e] += ps[e + w];
+        const float lsum = ps[0];
         // O holds PV of tiles 0..j-1 (the S MMA that signalled s_full was issued
         // after them); rescale it before this tile's PV is issued.
         if (warp_rescale && j > 0) {
