@@ -182,18 +182,19 @@ __global__ void __launch_bounds__(DkdvCfg<D>::THREADS, 1)
     {  // whole warp, warp-uniform values; one elected lane issues each MMA / commit
       constexpr uint32_t IDESC_T = idesc_bf16(128, C::BQ, false, false);  // S^T, dP^T: M=128 keys, N=64 queries
       constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);        // dV, dK: B operand MN-major
+      // S^T / dP^T: K = d; A (keys) and B (queries) K-major in shared memory.
       auto issue_t = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss_warp(d_tmem, sdesc_sw128(a_smem + (kk >> 2) * C::KCHUNK + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(b_smem + (kk >> 2) * C::QCHUNK + (kk & 3) * 32, 16, 1024), IDESC_T,
-                 kk > 0 ? 1u : 0u);
+        const uint32_t hi = sdesc_hi(1024);
+        const uint64_t a0 = sdesc_make(sdesc_lo(a_smem, 16), hi), b0 = sdesc_make(sdesc_lo(b_smem, 16), hi);
+        if (D == 128)
+          mma_ss_k128(d_tmem, a0, sdesc_make(sdesc_lo(a_smem + C::KCHUNK, 16), hi), b0,
+                      sdesc_make(sdesc_lo(b_smem + C::QCHUNK, 16), hi), IDESC_T, 0u);
+        else
+          mma_ss_k64(d_tmem, a0, b0, IDESC_T, 0u);
       };
+      // dV / dK: K = 64 queries; A (P^T or dS^T) from tensor memory, B MN-major.
       auto issue_g = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts_warp(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 16 * 128, C::QCHUNK, 1024), IDESC_G,
-                 (acc || kk > 0) ? 1u : 0u);
+        mma_ts_k64(d_tmem, a_tmem, sdesc_make(sdesc_lo(b_smem, C::QCHUNK), sdesc_hi(1024)), IDESC_G, acc ? 1u : 0u);
       };
       bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_KV_FULL, 0, BW_MMA_KV));
       tc_fence_after();
@@ -407,12 +408,15 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
     {  // whole warp, warp-uniform values; one elected lane issues each MMA / commit
       constexpr uint32_t IDESC_S = idesc_bf16(128, C::BK, false, false);  // S, dP: M=128 queries, N=64 keys
       constexpr uint32_t IDESC_Q = idesc_bf16(128, D, false, true);       // dQ: B (K tile) MN-major
+      // S / dP: K = d; A (queries) and B (keys) K-major in shared memory.
       auto issue_s = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss_warp(d_tmem, sdesc_sw128(a_smem + (kk >> 2) * C::QCHUNK + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(b_smem + (kk >> 2) * C::KCHUNK + (kk & 3) * 32, 16, 1024), IDESC_S,
-                 kk > 0 ? 1u : 0u);
+        const uint32_t hi = sdesc_hi(1024);
+        const uint64_t a0 = sdesc_make(sdesc_lo(a_smem, 16), hi), b0 = sdesc_make(sdesc_lo(b_smem, 16), hi);
+        if (D == 128)
+          mma_ss_k128(d_tmem, a0, sdesc_make(sdesc_lo(a_smem + C::QCHUNK, 16), hi), b0,
+                      sdesc_make(sdesc_lo(b_smem + C::KCHUNK, 16), hi), IDESC_S, 0u);
+        else
+          mma_ss_k64(d_tmem, a0, b0, IDESC_S, 0u);
       };
       bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_FULL, 0, BQ_MMA_Q));
       tc_fence_after();
@@ -429,11 +433,10 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
           const int pit = it - 1, pst = pit % C::ST, pb = pit & 1;
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BQ_MMA_P)))) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            mma_ts_warp(tmem + C::TM_DQ, tmem + C::TM_DP + pb * 64 + kk * 8,
-                   sdesc_sw128(sK + pst * C::K_TILE + kk * 16 * 128, C::KCHUNK, 1024), IDESC_Q,
-                   (pit > 0 || kk > 0) ? 1u : 0u);
+          // dQ += dS K: K = 64 keys; dS from tensor memory, K tile MN-major.
+          mma_ts_k64(tmem + C::TM_DQ, tmem + C::TM_DP + pb * 64,
+                     sdesc_make(sdesc_lo(sK + pst * C::K_TILE, C::KCHUNK), sdesc_hi(1024)), IDESC_Q,
+                     pit > 0 ? 1u : 0u);
           tc_commit_warp(bars + 8 * (C::B_KV_EMPTY + pst));
         }
       }

@@ -204,6 +204,102 @@ __device__ __forceinline__ void tc_commit_warp(uint32_t bar) {
       : "memory");
 }
 
+// Grouped issue: one elect.sync, then the MMAs of a whole K loop.  A shared-
+// memory descriptor advances along K by adding to its start-address field
+// (16-byte units): +2 per K step of 16 bf16 inside a 128-byte row, and a new
+// 64-column chunk starts from its own base descriptor.  All lanes call these
+// with warp-uniform operands; the elected lane issues.
+//
+// K = 128, A and B K-major in shared memory (two 64-column chunks each).
+__device__ __forceinline__ void mma_ss_k128(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t b0, uint64_t b1,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 ax, bx;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "setp.eq.b32 t, %5, %5;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %5, p;\n\t"
+      "add.s64 ax, %1, 2;\n\tadd.s64 bx, %3, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %1, 4;\n\tadd.s64 bx, %3, 4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %1, 6;\n\tadd.s64 bx, %3, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %4, %5, t;\n\t"
+      "add.s64 ax, %2, 2;\n\tadd.s64 bx, %4, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %2, 4;\n\tadd.s64 bx, %4, 4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %2, 6;\n\tadd.s64 bx, %4, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %5, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// K = 64, A and B K-major in shared memory (one 64-column chunk).
+__device__ __forceinline__ void mma_ss_k64(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 ax, bx;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 ax, %1, 2;\n\tadd.s64 bx, %2, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 4;\n\tadd.s64 bx, %2, 4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 6;\n\tadd.s64 bx, %2, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// A from tensor memory (K-major, 8 columns of packed bf16 per K step of 16),
+// B MN-major in shared memory (16 rows of 128 bytes = +128 per K step).
+// K = 128 (8 steps).
+__device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 bx;\n\t.reg .b32 ax;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ax, %1, 8;\n\tadd.s64 bx, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 16;\n\tadd.s64 bx, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 24;\n\tadd.s64 bx, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 32;\n\tadd.s64 bx, %2, 512;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 40;\n\tadd.s64 bx, %2, 640;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 48;\n\tadd.s64 bx, %2, 768;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 56;\n\tadd.s64 bx, %2, 896;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// K = 64 (4 steps).
+__device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 bx;\n\t.reg .b32 ax;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ax, %1, 8;\n\tadd.s64 bx, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 16;\n\tadd.s64 bx, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 24;\n\tadd.s64 bx, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Warp-collective TMEM load, shape 32x32b: thread t of the warp reads lane
 // (32 * (warp % 4) + t) of the address's lane window, 32 consecutive columns.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

@@ -180,25 +180,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     {
       constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
-      // S = Q_t K_j^T: D/16 steps of K = 16 (32 bytes inside a 128-byte row; the
-      // next 64-column chunk starts CHUNK bytes later).
+      // S = Q_t K_j^T: K = d in steps of 16 (one 8- or 4-MMA group).
       auto issue_s = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
         const uint32_t hi = sdesc_hi(1024);
-#pragma unroll 1
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss_warp(d_tmem, sdesc_make(sdesc_lo(a_smem + off, 16), hi), sdesc_make(sdesc_lo(b_smem + off, 16), hi),
-                 IDESC_S, kk > 0 ? 1u : 0u);
-        }
+        const uint64_t a0 = sdesc_make(sdesc_lo(a_smem, 16), hi), b0 = sdesc_make(sdesc_lo(b_smem, 16), hi);
+        if (D == 128)
+          mma_ss_k128(d_tmem, a0, sdesc_make(sdesc_lo(a_smem + C::CHUNK, 16), hi), b0,
+                      sdesc_make(sdesc_lo(b_smem + C::CHUNK, 16), hi), IDESC_S, 0u);
+        else
+          mma_ss_k64(d_tmem, a0, b0, IDESC_S, 0u);
       };
-      // O_t += P_t V_j: 8 steps of 16 keys; P_t from tensor memory (8 columns of
-      // packed bf16 per step), V_j MN-major (16 rows of 128 bytes per step).
+      // O_t += P_t V_j: 8 steps of 16 keys; P_t from tensor memory, V_j MN-major.
       auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
-        const uint32_t hi = sdesc_hi(1024);
-#pragma unroll 1
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts_warp(d_tmem, p_tmem + kk * 8, sdesc_make(sdesc_lo(v_smem + kk * 16 * 128, C::CHUNK), hi), IDESC_PV,
-                 (acc || kk > 0) ? 1u : 0u);
+        mma_ts_k128(d_tmem, p_tmem, sdesc_make(sdesc_lo(v_smem, C::CHUNK), sdesc_hi(1024)), IDESC_PV,
+                    acc ? 1u : 0u);
       };
       uint32_t kv_it = 0, q_it = 0, unit_it = 0;
       uint32_t p_ph0 = 0, p_ph1 = 0;
@@ -225,7 +220,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int j = 0; j < nk1 && ok; ++j) {
           const uint32_t it = kv_it + j;
           const int s = it % C::ST;
+          const bool more = j + 1 < nk1;
+          const int sn = (it + 1) % C::ST;
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_V_FULL + s), (it / C::ST) & 1, FW_MMA_V)))) break;
+          if (more && !(ok = __all_sync(0xffffffffu,
+                                        mbar_wait(bars + 8 * (C::B_K_FULL + sn), ((it + 1) / C::ST) & 1, FW_MMA_K))))
+            break;
           tc_fence_after();
           if (j < nk0) {
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + 0), p_ph0, FW_MMA_P)))) break;
@@ -235,11 +235,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             issue_pv(tmem + C::TM_O0, tmem + C::TM_S0, sV + s * C::KV_TILE, j > 0);
             if (j == nk0 - 1) tc_commit_warp(bars + 8 * (C::B_O_FULL + 0));
           }
-          const bool more = j + 1 < nk1;
-          const int sn = (it + 1) % C::ST;
           if (more) {
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_K_FULL + sn), ((it + 1) / C::ST) & 1, FW_MMA_K)))) break;
-            tc_fence_after();
             if (j + 1 < nk0) {
               issue_s(tmem + C::TM_S0, sQ, sK + sn * C::KV_TILE);
               tc_commit_warp(bars + 8 * (C::B_S_FULL + 0));
