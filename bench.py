@@ -164,6 +164,31 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------------------
+# cross-rank pieces (no GPU needed; tested with gloo ranks on the CPU)
+# ---------------------------------------------------------------------------
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank contributes, every rank gets the max."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Weak scaling: every rank runs its own batch, so the job did world x the
+    work of one rank in the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch."""
+    return base_seed + rank
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def run_ours(args, rank, world, local_rank):
@@ -178,7 +203,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     w = WORKLOADS[WORKLOAD]
     B, H, N, d = w.B, w.H, w.N, w.d
-    q, k, v, do = attention_inputs(B, H, N, d, seed=w.seed + rank)
+    q, k, v, do = attention_inputs(B, H, N, d, seed=rank_seed(w.seed, rank))
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o = torch.empty_like(qd)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -228,13 +253,6 @@ def run_ours(args, rank, world, local_rank):
                     "fa_bwd_dq_kernel": [e[3].elapsed_time(e[4]) for e in kev]}
         return total, kern
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # warm-up (also the status check: a kernel timeout would show here)
     for _ in range(max(args.warmup, 3)):
         fwd(False); bwd(False); fwd(True); bwd(True)
@@ -251,10 +269,10 @@ def run_ours(args, rank, world, local_rank):
         fwd_ms, _ = timed(lambda: fwd(False), args.steps)
         fwdc_ms, _ = timed(lambda: fwd(True), args.steps)
         stepc_ms, _ = timed(lambda: (fwd(True), bwd(True)), args.steps)
-    main_ms = max_over_ranks(main_ms)
-    fwd_ms = max_over_ranks(fwd_ms)
-    fwdc_ms = max_over_ranks(fwdc_ms)
-    stepc_ms = max_over_ranks(stepc_ms)
+    main_ms = max_over_ranks(main_ms, world, dev)
+    fwd_ms = max_over_ranks(fwd_ms, world, dev)
+    fwdc_ms = max_over_ranks(fwdc_ms, world, dev)
+    stepc_ms = max_over_ranks(stepc_ms, world, dev)
     rc = fa.sync_status(dev)
     if rc != fa.FA_OK:
         raise RuntimeError(f"library status {fa.status_string(rc)}")
@@ -275,13 +293,13 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e2e_ms, _ = timed(e2e_step, max(3, args.steps // 4))
     e2e_steps = max(3, args.steps // 4)
-    e2e_ms = max_over_ranks(e2e_ms)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
     d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
 
     peaks = _peaks()
     step_flops = f_nc + b_nc
-    value = world * step_flops * args.steps / (main_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, step_flops, args.steps, main_ms)
     # per-kernel live durations (rank-local) and the dominant kernel's roofline
     kavg = {n: sum(v) / len(v) for n, v in kern.items()}
     per_kernel_flops = {  # dense MMA work each kernel performs

@@ -3,10 +3,13 @@
 #include <math.h>
 #include <mutex>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd2.cuh"
 
 namespace {
 
@@ -53,6 +56,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   int checked = 0;  // 0 unknown, 1 supported, -1 unsupported
   int sms = 0;
+  int pair_clusters[2] = {0, 0};  // co-resident 2-CTA clusters of the paired forward kernel (non-causal, causal)
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -64,7 +68,7 @@ bool set_smem(Kern k, int bytes) {
 
 // Returns FA_OK and the SM count if the current device is sm_100 and the
 // kernels' shared-memory limits are set on it.
-int device_ready(int* sms) {
+int device_ready(int* sms, int* pair_clusters = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_UNSUPPORTED_DEVICE;
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED_DEVICE;
@@ -95,12 +99,35 @@ int device_ready(int* sms) {
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<64, true>, fa::DqCfg<64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, false>, fa::DqCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, true>, fa::DqCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_2sm_kernel<false>, fa::Fwd2Cfg::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_2sm_kernel<true>, fa::Fwd2Cfg::SMEM_BYTES);
+    for (int c = 0; c < 2 && ok; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * n, 1, 1);
+      cfg.blockDim = dim3(fa::Fwd2Cfg::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = fa::Fwd2Cfg::SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      const cudaError_t e = c ? cudaOccupancyMaxActiveClusters(&clusters, fa::fa_fwd_2sm_kernel<true>, &cfg)
+                              : cudaOccupancyMaxActiveClusters(&clusters, fa::fa_fwd_2sm_kernel<false>, &cfg);
+      di.pair_clusters[c] = (e == cudaSuccess) ? clusters : 0;
+    }
     cudaGetLastError();
     di.checked = ok ? 1 : -1;
     di.sms = n;
   }
   if (di.checked != 1) return FA_ERR_UNSUPPORTED_DEVICE;
   *sms = di.sms;
+  if (pair_clusters) {
+    pair_clusters[0] = di.pair_clusters[0];
+    pair_clusters[1] = di.pair_clusters[1];
+  }
   return FA_OK;
 }
 
@@ -192,8 +219,8 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   if (overlaps(ro, rq) || overlaps(ro, rk) || overlaps(ro, rv) || overlaps(ro, rl) || overlaps(rl, rq) ||
       overlaps(rl, rk) || overlaps(rl, rv))
     return FA_ERR_INVALID_ARG;
-  int sms = 0;
-  if ((rc = device_ready(&sms))) return rc;
+  int sms = 0, pair_clusters[2] = {0, 0};
+  if ((rc = device_ready(&sms, pair_clusters))) return rc;
   if (!is_device_ptr(Q) || !is_device_ptr(K) || !is_device_ptr(V) || !is_device_ptr(O) || !is_device_ptr(LSE))
     return FA_ERR_UNSUPPORTED_DEVICE;
   const int BH = B * H;
@@ -201,6 +228,28 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   if (!make_map(&mq, Q, BH, N, d, 128) || !make_map(&mk, K, BH, N, d, 128) || !make_map(&mv, V, BH, N, d, 128))
     return encode_failed();
   clear_stale_error();
+  // d = 128 non-causal: the paired (2-SM) kernel (faster there); causal and
+  // d = 64 run the 1-SM kernel.  FA_FWD_PAIR=0 / =1 forces one or the other
+  // for d = 128 (comparisons and tests).
+  const char* pair_env = getenv("FA_FWD_PAIR");
+  const int clusters = pair_clusters[causal ? 1 : 0];
+  bool use_pair = d == 128 && clusters > 0 && !causal;
+  if (pair_env && strcmp(pair_env, "0") == 0) use_pair = false;
+  if (pair_env && strcmp(pair_env, "1") == 0) use_pair = d == 128 && clusters > 0;
+  if (use_pair) {
+    CUtensorMap mkh;
+    if (!make_map(&mkh, K, BH, N, d, 64)) return encode_failed();
+    const int nqp = (N + 255) / 256, punits = BH * nqp;
+    const int pairs = punits < clusters ? punits : clusters;
+    const float sl2p = sc * fa::kLog2e;
+    cudaStream_t sp = static_cast<cudaStream_t>(stream);
+    auto* op = static_cast<__nv_bfloat16*>(O);
+    if (causal)
+      fa::fa_fwd_2sm_kernel<true><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p);
+    else
+      fa::fa_fwd_2sm_kernel<false><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p);
+    return launch_status();
+  }
   const int nqt = (N + 127) / 128, units = BH * ((nqt + 1) / 2);
   const int grid = units < sms ? units : sms;
   const float sl2 = sc * fa::kLog2e;

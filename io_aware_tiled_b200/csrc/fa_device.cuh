@@ -88,6 +88,58 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 }
 
 // ---------------------------------------------------------------------------
+// clusters of two CTAs (the 2-SM tensor-core form)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared_to_rank(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
+               "r"(bytes)
+               : "memory");
+}
+// Non-blocking test (test_wait): a thread suspended in try_wait is not woken
+// promptly by an arrival from the peer CTA, so cluster-scope waits poll.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+// Bounded wait on a local barrier that the peer CTA also arrives on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, unsigned int where) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 256; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(kErrTimeout, where);
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // register reallocation between warpgroups (warpgroup-wide; the sum over the
 // CTA must stay within the registers it was launched with)
 // ---------------------------------------------------------------------------
@@ -121,6 +173,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// 3-D tiled load issued by either CTA of a pair, completing on the barrier at
+// `bar_cluster_addr` (the leader CTA's barrier); no multicast.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 
@@ -296,6 +359,79 @@ __device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uin
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t"
       "add.s32 ax, %1, 24;\n\tadd.s64 bx, %2, 384;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ax], bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 2-SM forms (cta_group::2): issued by the leader CTA of a pair; A and D rows
+// are split between the two CTAs (M/2 each), B's N columns likewise.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive once on the barrier at this offset in every CTA of `cta_mask` when all
+// prior tcgen05 operations of this thread complete.
+__device__ __forceinline__ void tc_commit_pair_warp(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_ss_k128(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t b0, uint64_t b1,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 ax, bx;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "setp.eq.b32 t, %5, %5;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %3, %5, p;\n\t"
+      "add.s64 ax, %1, 2;\n\tadd.s64 bx, %3, 2;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %1, 4;\n\tadd.s64 bx, %3, 4;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %1, 6;\n\tadd.s64 bx, %3, 6;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %2, %4, %5, t;\n\t"
+      "add.s64 ax, %2, 2;\n\tadd.s64 bx, %4, 2;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %2, 4;\n\tadd.s64 bx, %4, 4;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], ax, bx, %5, t;\n\t"
+      "add.s64 ax, %2, 6;\n\tadd.s64 bx, %4, 6;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], ax, bx, %5, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma2_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 bx;\n\t.reg .b32 ax;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ax, %1, 8;\n\tadd.s64 bx, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 16;\n\tadd.s64 bx, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 24;\n\tadd.s64 bx, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 32;\n\tadd.s64 bx, %2, 512;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 40;\n\tadd.s64 bx, %2, 640;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 48;\n\tadd.s64 bx, %2, 768;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 56;\n\tadd.s64 bx, %2, 896;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b0), "r"(idesc), "r"(accumulate)
       : "memory");
 }

@@ -315,3 +315,24 @@ def test_wait_timeout_is_reported_and_context_survives():
     o, lse = _run_fwd(q, k, v, False)
     ro, rl = oracle.forward(f64(q), f64(k), f64(v), False, 1 / 8)
     check_o(f64(o), ro, "after timeout")
+
+
+PAIR_CASES = [(1, 3, 1000, True), (1, 3, 1000, False), (2, 2, 300, True), (1, 3, 333, True),
+              (1, 1, 129, False), (1, 1, 1, True), (1, 2, 2048, False), (1, 1, 640, True)]
+
+
+@pytest.mark.parametrize("B,H,N,causal", PAIR_CASES)
+def test_both_forward_kernels_for_d128(B, H, N, causal, monkeypatch):
+    """d = 128 has two forward kernels: one SM per CTA, and CTA pairs (2-SM
+    MMAs).  FA_FWD_PAIR=0 / =1 forces either; both match the oracle, ragged
+    tails and query tiles past N included."""
+    d = 128
+    q, k, v, _ = attention_inputs(B, H, N, d, seed=21 + N, with_do=False)
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), causal, 1 / d ** 0.5)
+    for mode in ("0", "1"):
+        monkeypatch.setenv("FA_FWD_PAIR", mode)
+        o, lse = _run_fwd(q, k, v, causal)
+        what = f"{'paired' if mode == '1' else 'one-SM'} {B,H,N} causal={causal}"
+        check_o(f64(o), ro, what)
+        check_lse(f64(lse), rl, what)
+    monkeypatch.delenv("FA_FWD_PAIR")
