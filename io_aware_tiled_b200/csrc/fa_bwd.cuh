@@ -114,9 +114,13 @@ __global__ void __launch_bounds__(DkdvCfg<D>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Block order: head-major without a mask (the blocks resident together
+  // share one head's Q and dO in L2); with the causal mask, the longest key
+  // tiles (the first ones) of every head come first, so the last wave is short.
   const int NKT = (N + C::BK - 1) / C::BK;
-  const int bh = blockIdx.x / NKT;
-  const int kt = blockIdx.x - bh * NKT;
+  const int BHg = gridDim.x / NKT;
+  const int bh = CAUSAL ? blockIdx.x % BHg : blockIdx.x / NKT;
+  const int kt = CAUSAL ? blockIdx.x / BHg : blockIdx.x - bh * NKT;
   const int NQT = (N + C::BQ - 1) / C::BQ;
   const int i0 = CAUSAL ? (kt * C::BK) / C::BQ : 0;  // first query tile that sees these keys
   const int nt = NQT - i0;                           // >= 1: the tile holding query kt*BK exists
@@ -355,9 +359,12 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Block order as in the dK/dV kernel: head-major without a mask, longest
+  // query tiles (the last ones) of every head first with it.
   const int NQT = (N + C::BQ - 1) / C::BQ;
-  const int bh = blockIdx.x / NQT;
-  const int qt = blockIdx.x - bh * NQT;
+  const int BHg = gridDim.x / NQT;
+  const int bh = CAUSAL ? blockIdx.x % BHg : blockIdx.x / NQT;
+  const int qt = CAUSAL ? NQT - 1 - blockIdx.x / BHg : blockIdx.x - bh * NQT;
   const int NKT = (N + C::BK - 1) / C::BK;
   const int nt = CAUSAL ? min(NKT, (qt * C::BQ + C::BQ - 1) / C::BK + 1) : NKT;
 

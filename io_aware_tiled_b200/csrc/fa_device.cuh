@@ -539,6 +539,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Index of the k-th work unit of a persistent worker w out of W: units are
+// dealt in rounds of W, left to right on even rounds and right to left on odd
+// ones ("serpentine").  With units sorted longest first this balances the
+// per-worker sums far better than plain round robin.
+__device__ __forceinline__ int serpentine_unit(int k, int w, int W) {
+  return k * W + ((k & 1) ? (W - 1 - w) : w);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -74,7 +74,8 @@ enum FwdWaitSite : unsigned int {
 
 // Unit order.  Non-causal: head-major, so the CTAs running at the same time
 // share a few heads' K and V in L2.  Causal: longest units (last query pairs)
-// first across all heads, so the persistent CTAs finish together.
+// first across all heads, dealt in serpentine order (serpentine_unit), so the
+// persistent CTAs finish together.
 __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool causal, int& bh, int& qp) {
   if (causal) {
     const int r = u / BH;
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t kv_it = 0, q_it = 0;
-      for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      for (int k = 0, u = blockIdx.x; u < units; u = serpentine_unit(++k, blockIdx.x, gridDim.x)) {
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
         const int nk1 = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       };
       uint32_t kv_it = 0, q_it = 0, unit_it = 0;
       uint32_t p_ph0 = 0, p_ph1 = 0;
-      for (int u = blockIdx.x; u < units; u += gridDim.x, ++unit_it) {
+      for (int k = 0, u = blockIdx.x; u < units; u = serpentine_unit(++k, blockIdx.x, gridDim.x), ++unit_it) {
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
         (void)bh;
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const uint32_t bar_o = bars + 8 * (C::B_O_FULL + wg), bar_oe = bars + 8 * (C::B_O_EMPTY + wg);
     uint32_t s_it = 0, o_it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int k = 0, u = blockIdx.x; u < units && ok; u = serpentine_unit(++k, blockIdx.x, gridDim.x)) {
       int bh, qp;
       fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
       const int qt = 2 * qp + wg;

@@ -22,9 +22,11 @@
 //     arrival costs hundreds of nanoseconds, too much for 128 threads on the
 //     critical path); in CTA 1 a relay warp forwards each completed phase to
 //     the leader with a single remote arrival.
-//   * Softmax: one thread per row, base 2, O rescaled only when a row max grows
-//     by more than 2^8; before rescaling, the softmax waits for the previous PV
-//     (an "O done" barrier committed after every PV).
+//   * Softmax: two warpgroups per CTA split every row's 128 scores (64 each);
+//     they exchange partial row maxima through shared memory once per step and
+//     combine row sums only at the end.  Base 2; O (each warpgroup its half of
+//     the columns) is rescaled only when a row max grows by more than 2^8, after
+//     waiting for the previous PV (an "O done" barrier committed after every PV).
 #pragma once
 
 #include "fa_device.cuh"
@@ -52,10 +54,13 @@ struct Fwd2Cfg {
                        B_O_EMPTY = B_O_DONE + 2;  // O_DONE[2]: PV of tile g commits to O_DONE[g % 2]
   static constexpr int NUM_BARS = B_O_EMPTY + 1;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
+  static constexpr int OFF_XCH = OFF_TMEM_SLOT + 16;  // max exchange [2 steps][2 halves][128] + sums [2][128]
+  static constexpr int SMEM_BYTES = OFF_XCH + 6 * 128 * 4 + 1024;
   static constexpr uint32_t TM_O = 384;          // S buffer b at column 128 * b
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 256;            // warp 0 loads, warp 1 MMA (leader), warps 4-7 softmax
+  // warp 0 loads, warp 1 MMA (leader) or relay (peer), warps 4-7 and 8-11: the
+  // softmax warpgroups of the low and the high 64 columns
+  static constexpr int THREADS = 384;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
   static constexpr uint16_t BOTH = 0x3;          // multicast mask: both CTAs of the pair
 };
@@ -109,9 +114,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
       mbar_init(bar(C::B_V_FULL + s), 1);
       mbar_init(bar(C::B_V_EMPTY + s), 1);
     }
-    // P and O-empty: the 128 local softmax threads, plus on the leader the
+    // P and O-empty: the 256 local softmax threads, plus on the leader the
     // relay's one arrival for CTA 1
-    const uint32_t cnt = rank == 0 ? 129u : 128u;
+    const uint32_t cnt = rank == 0 ? 257u : 256u;
     for (int b = 0; b < C::NS; ++b) {
       mbar_init(bar(C::B_S_FULL + b), 1);
       mbar_init(bar(C::B_P_FULL + b), cnt);
@@ -145,7 +150,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     // ------------------------------------------------------------ loads (both CTAs)
     if (lane == 0) {
       uint32_t kv_it = 0, q_it = 0;
-      for (int u = pair; u < units; u += npairs) {
+      for (int k = 0, u = pair; u < units; u = serpentine_unit(++k, pair, npairs)) {
         int bh, qp;
         fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
         const int nk = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
@@ -194,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
       tc_commit_pair_warp(bar(C::B_K_EMPTY + s), C::BOTH);
       return true;
     };
-    for (int u = pair; u < units && ok; u += npairs, ++unit_it) {
+    for (int k = 0, u = pair; u < units && ok; u = serpentine_unit(++k, pair, npairs), ++unit_it) {
       int bh, qp;
       fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
       (void)bh;
@@ -236,7 +241,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     // leader's, one remote arrival per phase.
     if (lane == 0) {
       uint32_t g = 0, unit_it = 0;
-      for (int u = pair; u < units; u += npairs, ++unit_it) {
+      for (int k = 0, u = pair; u < units; u = serpentine_unit(++k, pair, npairs), ++unit_it) {
         int bh, qp;
         fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
         (void)bh;
@@ -257,20 +262,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
       }
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax warpgroup (both CTAs)
+    // ------------------------------------------------------------ softmax warpgroups (both CTAs)
+    const int h = (warp - 4) >> 2;           // which 64 of the 128 columns
     const int sp = warp & 3;
-    const int r = sp * 32 + lane;
+    const int r = sp * 32 + lane;            // the row (TMEM lane) this thread shares with its partner
     const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
-    const uint32_t tO = tmem + lane_off + C::TM_O;
+    const uint32_t tO = tmem + lane_off + C::TM_O + 64 * h;  // this warpgroup's half of O
+    float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
+    float* xmax = xch;                        // [step & 1][half][row]
+    float* xsum = xch + 4 * 128;              // [half][row]
     uint32_t s_it = 0;
     bool ok = true;
-    for (int u = pair; u < units && ok; u += npairs) {
+    for (int k = 0, u = pair; u < units && ok; u = serpentine_unit(++k, pair, npairs)) {
       int bh, qp;
       fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
       const int qt = 2 * qp + static_cast<int>(rank);
       const int nk = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
       const int row = qt * C::BM + r;
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f;  // l: this thread's partial row sum
       for (int j = 0; j < nk; ++j) {
         const uint32_t g = s_it;  // global tile index of this CTA pair
         const int b = g % C::NS;
@@ -279,19 +288,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
         if (!(ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(C::B_S_FULL + b), sph, F2_SM_S)))) break;
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + 128 * b;
-        uint32_t sr[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        uint32_t sr[64];
+        tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_ld_wait();
+        reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        float s[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-        float s[128];
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
+        const int kbase = j * C::BN + 64 * h;
+        if ((CAUSAL && j * C::BN + C::BN - 1 > qt * C::BM) || j * C::BN + C::BN > N) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-        const int kbase = j * C::BN;
-        if ((CAUSAL && kbase + C::BN - 1 > qt * C::BM) || kbase + C::BN > N) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
+          for (int c = 0; c < 64; ++c) {
             const int key = kbase + c;
             if (key >= N || (CAUSAL && key > row)) s[c] = -INFINITY;
           }
@@ -300,14 +309,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) pm[e] = s[e];
 #pragma unroll
-        for (int c = 8; c < 128; c += 8)
+        for (int c = 8; c < 64; c += 8)
 #pragma unroll
           for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
 #pragma unroll
         for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
           for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
-        const float m_new = fmaxf(m_ref, pm[0] * scale_log2);
+        // Row max across the two halves.  The exchange slot alternates with the
+        // step, so a slot is rewritten only after the partner has passed the
+        // next barrier, i.e. after it read this step's value.  Both halves
+        // then hold the same max, hence the same m and rescale decisions.
+        float* slot = xmax + (j & 1) * 256;
+        slot[h * 128 + r] = pm[0];
+        named_bar_sync(1, 256);
+        const float mx = fmaxf(pm[0], slot[(1 - h) * 128 + r]);
+        // Both halves have loaded their S before that barrier, so from here on
+        // P may be written over S's columns.
+        const float m_new = fmaxf(m_ref, mx * scale_log2);
         const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
         const bool warp_rescale = __any_sync(0xffffffffu, need);
         const float alpha = need ? ex2(m_ref - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
@@ -319,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
         const float neg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
@@ -328,7 +347,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
             ps[c & 7] += p0 + p1;
             p[c] = pack_bf16(p0, p1);
           }
-          tmem_st16(tS + ch * 16, p);
+          tmem_st16(tS + 32 * h + ch * 16, p);  // keys 64h.. -> packed columns 32h..
         }
 #pragma unroll
         for (int w = 4; w > 0; w >>= 1)
@@ -348,17 +367,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
         if (!ok) break;
         if (j > 0 && warp_rescale) {
           tc_fence_after();
-          {
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tO + c * 32, o);
-              tmem_ld_wait();
-              reg_fence(o);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_ld_wait();
+            reg_fence(o);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tO + c * 32, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c * 32, o);
           }
         }
         tmem_st_wait();
@@ -379,10 +396,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
         if (!ok) break;
       }
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = O + (static_cast<size_t>(bh) * N + row) * D;
+      xsum[h * 128 + r] = l;
+      named_bar_sync(1, 256);
+      const float l_row = l + xsum[(1 - h) * 128 + r];
+      const float inv_l = 1.f / l_row;
+      __nv_bfloat16* orow = O + (static_cast<size_t>(bh) * N + row) * D + 64 * h;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_ld_wait();
@@ -400,7 +420,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
           }
         }
       }
-      if (row < N) LSE[static_cast<size_t>(bh) * N + row] = (m_ref + __log2f(l)) * kLn2;
+      if (h == 0 && row < N) LSE[static_cast<size_t>(bh) * N + row] = (m_ref + __log2f(l_row)) * kLn2;
       tc_fence_before();
       mbar_arrive(bar(C::B_O_EMPTY));
     }
