@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 _ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -57,25 +58,73 @@ def _flops(B, H, N, d, causal):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event reasons sampled during the timed region.
+
+    NVML in a background thread every 5 ms (the timed region lasts well under
+    a second); `nvidia-smi -lms 100` when NVML is not importable.  The thread
+    takes its first sample before __enter__ returns."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                   ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device):
+        self.device = device
         self.proc = None
         self.out = None
+        self.samples = []      # (sm_mhz, reason bitmask)
+        self.sm_max = None
+        self.thread = None
+        self.stop = threading.Event()
+
+    def _nvml_handle(self, nvml):
+        import torch
+        p = torch.cuda.get_device_properties(self.device)
+        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        try:
+            return nvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except nvml.NVMLError:
+            return nvml.nvmlDeviceGetHandleByPciBusId(bus[4:])
 
     def __enter__(self):
         try:
+            import pynvml as nvml
+            nvml.nvmlInit()
+            h = self._nvml_handle(nvml)
+            self.sm_max = float(nvml.nvmlDeviceGetMaxClockInfo(h, nvml.NVML_CLOCK_SM))
+            first = threading.Event()
+
+            def loop():
+                while True:
+                    try:
+                        self.samples.append((float(nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM)),
+                                             int(nvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except nvml.NVMLError:
+                        pass
+                    first.set()
+                    if self.stop.wait(0.005):
+                        return
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            first.wait(2.0)
+            return self
+        except Exception:  # no NVML: fall back to nvidia-smi
+            self.thread = None
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "-i", str(self.device.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -86,6 +135,14 @@ class ClockSampler:
         return False
 
     def summary(self):
+        if self.samples:
+            sm = [c for c, _ in self.samples]
+            mask = 0
+            for _, m in self.samples:
+                mask |= m
+            reasons = sorted(n for n, bit in self.REASON_BITS if mask & bit)
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.sm_max, "reasons": reasons,
+                    "samples": len(sm), "sm_mhz_min": min(sm), "source": "nvml, 5 ms"}
         if not self.out:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         sm, smax, reasons = [], None, set()
@@ -103,7 +160,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 100 ms"}
 
 
 # ---------------------------------------------------------------------------
@@ -189,6 +246,43 @@ def rank_seed(base_seed: int, rank: int) -> int:
 
 
 # ---------------------------------------------------------------------------
+# DRAM traffic from ncu
+# ---------------------------------------------------------------------------
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of each kernel,
+# captured with `python bench.py --ncu-case fwd|bwd` (B=4, H=16, N=4096,
+# d=128, non-causal: 64 heads) and divided by the 64 heads; the summaries sit
+# in profiles/.  Each kernel reads its inputs once per head, so the traffic of
+# the bench's 32-head launch is the per-head figure x 32.  SOURCES_SHA is the
+# sha256 of the kernel sources at capture time: once they change the figures
+# no longer describe the kernels and traffic is reported as null.
+NCU_TRAFFIC_PER_HEAD = {
+    "fa_fwd_2sm_kernel": (201.413376e6 + 49.094656e6) / 64,
+    "fa_bwd_dkdv_kernel": (270.878720e6 + 103.970816e6) / 64,
+    "fa_bwd_dq_kernel": (270.584576e6 + 51.742208e6) / 64,
+}
+NCU_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_device.cuh", "fa_fwd.cuh", "fa_fwd2.cuh")
+NCU_SOURCES_SHA = "c6d45be6f17046b72e39a06805a2283f364c0f75bcb892c75b6f5959c9e26608"
+
+
+def kernel_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    root = os.path.join(os.path.dirname(os.path.abspath(__file__)), "io_aware_tiled_b200", "csrc")
+    for name in NCU_SOURCES:
+        with open(os.path.join(root, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic_per_launch(heads: int) -> dict:
+    """DRAM bytes per launch for `heads` (B*H) heads, by kernel name; empty
+    when the kernel sources changed since the capture."""
+    if kernel_sources_sha() != NCU_SOURCES_SHA:
+        return {}
+    return {n: b * heads for n, b in NCU_TRAFFIC_PER_HEAD.items()}
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def run_ours(args, rank, world, local_rank):
@@ -223,6 +317,8 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
+    fwd_name = fa.forward_kernel_name(d, False)
+
     def timed(fn, steps, per_kernel=False):
         """Run fn `steps` times, L2 flushed before each; returns total ms and
         per-kernel ms lists when per_kernel (forward + the three backward kernels)."""
@@ -247,7 +343,7 @@ def run_ours(args, rank, world, local_rank):
         total = sum(a.elapsed_time(b) for a, b in ev)
         kern = None
         if per_kernel:
-            kern = {"fa_fwd_kernel": [e[0].elapsed_time(e[1]) for e in kev],
+            kern = {fwd_name: [e[0].elapsed_time(e[1]) for e in kev],
                     "fa_bwd_preprocess_kernel": [e[1].elapsed_time(e[2]) for e in kev],
                     "fa_bwd_dkdv_kernel": [e[2].elapsed_time(e[3]) for e in kev],
                     "fa_bwd_dq_kernel": [e[3].elapsed_time(e[4]) for e in kev]}
@@ -263,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
     f_nc, b_nc = _flops(B, H, N, d, False)
     f_c, b_c = _flops(B, H, N, d, True)
 
-    clocks = ClockSampler(dev.index if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    clocks = ClockSampler(dev)
     with clocks:
         main_ms, kern = timed(None, args.steps, per_kernel=True)
         fwd_ms, _ = timed(lambda: fwd(False), args.steps)
@@ -303,23 +399,25 @@ def run_ours(args, rank, world, local_rank):
     # per-kernel live durations (rank-local) and the dominant kernel's roofline
     kavg = {n: sum(v) / len(v) for n, v in kern.items()}
     per_kernel_flops = {  # dense MMA work each kernel performs
-        "fa_fwd_kernel": 4.0 * B * H * N * N * d,
+        fwd_name: 4.0 * B * H * N * N * d,
         "fa_bwd_dkdv_kernel": 8.0 * B * H * N * N * d,   # S^T, dP^T, dV, dK
         "fa_bwd_dq_kernel": 6.0 * B * H * N * N * d,     # S, dP, dQ
     }
+    traffic = ncu_traffic_per_launch(B * H)
     dom = max(kavg, key=kavg.get)
     peak = peaks["bf16_tflops"]
     if dom in per_kernel_flops:
         ach = per_kernel_flops[dom] / (kavg[dom] * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None, "peak_kind": f"bf16 burst, {peaks['source']}"}
+                "frac": ach / peak, "traffic": traffic.get(dom), "peak_kind": f"bf16 burst, {peaks['source']}"}
     else:
         bytes_pre = 2.0 * B * H * N * d * 2 + 4.0 * B * H * N
         ach = bytes_pre / (kavg[dom] * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_kind": f"hbm copy, {peaks['source']}"}
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic.get(dom), "peak_kind": f"hbm copy, {peaks['source']}"}
     kernels = {n: {"ms": kavg[n],
-                   "tflops": (per_kernel_flops[n] / (kavg[n] * 1e-3) / 1e12) if n in per_kernel_flops else None}
+                   "tflops": (per_kernel_flops[n] / (kavg[n] * 1e-3) / 1e12) if n in per_kernel_flops else None,
+                   "traffic": traffic.get(n)}
                for n in kavg}
     kernels["fa_bwd_preprocess_kernel"]["gbs"] = (2.0 * B * H * N * d * 2 + 4.0 * B * H * N) / (
         kavg["fa_bwd_preprocess_kernel"] * 1e-3) / 1e9

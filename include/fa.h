@@ -143,6 +143,16 @@ void fa_bwd_set_phase_events(void* e0, void* e1, void* e2, void* e3);
 const char* fa_status_string(int status);
 
 /*
+ * Name of the kernel fa_fwd launches on the current device for head size d
+ * and the given mask flag: "fa_fwd_2sm_kernel" (CTA pairs, d = 128 without
+ * the mask) or "fa_fwd_kernel".  The environment variable FA_FWD_PAIR=0 / =1
+ * forces the one or the other for d = 128.  NULL when d is not 64 or 128 or
+ * the device is not usable.  Static string, owned by the library.  For
+ * labelling timings and profiles; the paper has no counterpart.
+ */
+const char* fa_fwd_kernel_name(int d, int causal);
+
+/*
  * Fault-detection self test.  Launches one tiny kernel that waits on a
  * barrier nothing ever signals, with a wall-clock limit of `limit_us`
  * microseconds (1 .. 10,000,000).  The wait runs out, the kernel records

@@ -203,6 +203,24 @@ const char* fa_status_string(int status) {
   }
 }
 
+// d = 128 non-causal: the paired (2-SM) kernel (faster there); causal and
+// d = 64 run the 1-SM kernel.  FA_FWD_PAIR=0 / =1 forces one or the other for
+// d = 128 (comparisons and tests).  `clusters`: CTA pairs that fit at once.
+static bool fwd_use_pair(int d, int causal, int clusters) {
+  const char* pair_env = getenv("FA_FWD_PAIR");
+  bool use_pair = d == 128 && clusters > 0 && !causal;
+  if (pair_env && strcmp(pair_env, "0") == 0) use_pair = false;
+  if (pair_env && strcmp(pair_env, "1") == 0) use_pair = d == 128 && clusters > 0;
+  return use_pair;
+}
+
+const char* fa_fwd_kernel_name(int d, int causal) {
+  if (d != 64 && d != 128) return nullptr;
+  int sms = 0, pair_clusters[2] = {0, 0};
+  if (device_ready(&sms, pair_clusters)) return nullptr;
+  return fwd_use_pair(d, causal, pair_clusters[causal ? 1 : 0]) ? "fa_fwd_2sm_kernel" : "fa_fwd_kernel";
+}
+
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
            int causal, float scale, void* stream) {
   int rc = check_sizes(B, H, N, d);
@@ -228,15 +246,8 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   if (!make_map(&mq, Q, BH, N, d, 128) || !make_map(&mk, K, BH, N, d, 128) || !make_map(&mv, V, BH, N, d, 128))
     return encode_failed();
   clear_stale_error();
-  // d = 128 non-causal: the paired (2-SM) kernel (faster there); causal and
-  // d = 64 run the 1-SM kernel.  FA_FWD_PAIR=0 / =1 forces one or the other
-  // for d = 128 (comparisons and tests).
-  const char* pair_env = getenv("FA_FWD_PAIR");
   const int clusters = pair_clusters[causal ? 1 : 0];
-  bool use_pair = d == 128 && clusters > 0 && !causal;
-  if (pair_env && strcmp(pair_env, "0") == 0) use_pair = false;
-  if (pair_env && strcmp(pair_env, "1") == 0) use_pair = d == 128 && clusters > 0;
-  if (use_pair) {
+  if (fwd_use_pair(d, causal, clusters)) {
     CUtensorMap mkh;
     if (!make_map(&mkh, K, BH, N, d, 64)) return encode_failed();
     const int nqp = (N + 255) / 256, punits = BH * nqp;

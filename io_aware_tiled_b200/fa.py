@@ -71,6 +71,8 @@ def load_library(build_if_missing: bool = True):
         lib.fa_last_cuda_error.restype = i
         lib.fa_status_string.argtypes = [i]
         lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_fwd_kernel_name.argtypes = [i, i]
+        lib.fa_fwd_kernel_name.restype = ctypes.c_char_p
         lib.fa_bwd_set_phase_events.argtypes = [vp, vp, vp, vp]
         lib.fa_bwd_set_phase_events.restype = None
         lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
@@ -87,6 +89,15 @@ def header_functions() -> list[str]:
 
 def status_string(status: int) -> str:
     return load_library().fa_status_string(int(status)).decode()
+
+
+def forward_kernel_name(d: int, causal: bool) -> str:
+    """Name of the kernel `forward` launches on the current device for head
+    size d (fa_fwd_kernel_name)."""
+    name = load_library().fa_fwd_kernel_name(int(d), int(bool(causal)))
+    if name is None:
+        raise RuntimeError(f"no forward kernel for d={d} on this device")
+    return name.decode()
 
 
 def _stream_handle(device: torch.device):

@@ -24,7 +24,7 @@ def test_every_declared_symbol_is_exported(lib):
     names = fa.header_functions()
     assert set(names) == {"fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_sync_status", "fa_last_error_word",
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
-                          "fa_last_cuda_error", "fa_bwd_noalloc"}
+                          "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:

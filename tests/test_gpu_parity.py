@@ -336,3 +336,21 @@ def test_both_forward_kernels_for_d128(B, H, N, causal, monkeypatch):
         check_o(f64(o), ro, what)
         check_lse(f64(lse), rl, what)
     monkeypatch.delenv("FA_FWD_PAIR")
+
+
+def test_forward_kernel_name_follows_the_routing(monkeypatch):
+    """fa_fwd_kernel_name reports the kernel fa_fwd launches: CTA pairs for
+    d = 128 without the mask, one SM per CTA otherwise, FA_FWD_PAIR forcing
+    either for d = 128; no name for an unsupported head size."""
+    monkeypatch.delenv("FA_FWD_PAIR", raising=False)
+    assert fa.forward_kernel_name(128, False) == "fa_fwd_2sm_kernel"
+    assert fa.forward_kernel_name(128, True) == "fa_fwd_kernel"
+    assert fa.forward_kernel_name(64, False) == "fa_fwd_kernel"
+    assert fa.forward_kernel_name(64, True) == "fa_fwd_kernel"
+    monkeypatch.setenv("FA_FWD_PAIR", "0")
+    assert fa.forward_kernel_name(128, False) == "fa_fwd_kernel"
+    monkeypatch.setenv("FA_FWD_PAIR", "1")
+    assert fa.forward_kernel_name(128, True) == "fa_fwd_2sm_kernel"
+    assert fa.forward_kernel_name(64, True) == "fa_fwd_kernel"
+    with pytest.raises(RuntimeError):
+        fa.forward_kernel_name(96, False)
