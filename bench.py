@@ -365,6 +365,15 @@ def run_ours(args, rank, world, local_rank):
         fwd_ms, _ = timed(lambda: fwd(False), args.steps)
         fwdc_ms, _ = timed(lambda: fwd(True), args.steps)
         stepc_ms, _ = timed(lambda: (fwd(True), bwd(True)), args.steps)
+    # the standard (unfused) forward of the same batch, for the HBM-traffic
+    # comparison: S and P through HBM (outside the clock sampling window)
+    ws_unf = torch.empty(fa.unfused_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        fa.forward_unfused(qd, kd, vd, False, workspace=ws_unf, out=o, lse=lse)
+    unf_steps = max(3, args.steps // 4)
+    unf_ms, _ = timed(lambda: fa.forward_unfused(qd, kd, vd, False, workspace=ws_unf, out=o, lse=lse), unf_steps)
+    unf_ms = max_over_ranks(unf_ms, world, dev)
+    del ws_unf
     main_ms = max_over_ranks(main_ms, world, dev)
     fwd_ms = max_over_ranks(fwd_ms, world, dev)
     fwdc_ms = max_over_ranks(fwdc_ms, world, dev)
@@ -439,6 +448,13 @@ def run_ours(args, rank, world, local_rank):
                                "ms": fwdc_ms / args.steps},
                 "fwd_bwd_causal": {"tflops": world * (f_c + b_c) * args.steps / (stepc_ms * 1e-3) / 1e12,
                                    "ms": stepc_ms / args.steps},
+                # standard attention: S (fp16) and P (bf16) written and read
+                # once each through HBM; bytes per head as in the pages'
+                # table: Q, K, V, S, P read; S, P, O written
+                "fwd_unfused_noncausal": {
+                    "tflops": world * f_nc * unf_steps / (unf_ms * 1e-3) / 1e12, "ms": unf_ms / unf_steps,
+                    "algorithmic_gbs": world * B * H * (3 * N * d * 2 + 4 * N * N * 2 + N * d * 2 + N * 4)
+                    * unf_steps / (unf_ms * 1e-3) / 1e9},
             },
             "kernels": kernels,
             "roofline": roof,
@@ -463,8 +479,12 @@ def run_ncu_case(case: str, batch: int):
     q, k, v, do = (t.to(dev) for t in attention_inputs(batch, 16, 4096, 128, seed=0))
     causal = case.endswith("causal")
     o, lse = fa.forward(q, k, v, causal)
+    ws_unf = torch.empty(fa.unfused_workspace_bytes(*q.shape), dtype=torch.uint8, device=dev) \
+        if case == "fwd_unfused" else None
     for _ in range(2):
-        if case.startswith("fwd"):
+        if case == "fwd_unfused":
+            fa.forward_unfused(q, k, v, False, workspace=ws_unf, out=o, lse=lse)
+        elif case.startswith("fwd"):
             fa.forward(q, k, v, causal, out=o, lse=lse)
         else:
             fa.backward(q, k, v, o, do, lse, causal)
@@ -480,7 +500,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["fwd", "fwd_causal", "bwd", "bwd_causal"], default=None,
+    ap.add_argument("--ncu-case", choices=["fwd", "fwd_causal", "bwd", "bwd_causal", "fwd_unfused"], default=None,
                     help="run a few untimed launches for an ncu capture and exit")
     ap.add_argument("--ncu-batch", type=int, default=4)
     args = ap.parse_args(argv)

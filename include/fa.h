@@ -139,6 +139,27 @@ int fa_last_cuda_error(void);
  */
 void fa_bwd_set_phase_events(void* e0, void* e1, void* e2, void* e3);
 
+/*
+ * Standard (unfused) attention forward: the comparison column of the HBM
+ * access table in "FlashAttention分块计算优化Transformer显存效率", section 2.1
+ * (内存访问模式对比).  Computes the same O and LSE as fa_fwd, but writes the
+ * score matrix S = scale * Q K^T (fp16) to HBM, reads it back for a row
+ * softmax that writes P (bf16) over it, and reads P for O = P V.  Exists to
+ * measure the HBM traffic the tiled kernels avoid; every score is computed
+ * (the causal mask is applied in the softmax).
+ *
+ * Arguments as fa_fwd, plus `workspace`: caller-owned device memory of at
+ * least fa_fwd_unfused_workspace_bytes(B, H, N, d) bytes, 16-byte aligned,
+ * not overlapping any other argument; it holds S, then P, as [B*H][Nr][Nr]
+ * 16-bit elements, Nr = N rounded up to a multiple of 128.  Returns
+ * FA_ERR_WORKSPACE when it is missing, too small, misaligned or overlaps
+ * another argument, otherwise the same codes as fa_fwd.  Asynchronous on `stream`.  The 16-bit S limits LSE accuracy to
+ * about max|score| * 2^-11 (it is exact to 1e-3 for scores of magnitude < 2).
+ */
+size_t fa_fwd_unfused_workspace_bytes(int B, int H, int N, int d);
+int fa_fwd_unfused(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+                   int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Human-readable name of an fa_status value (static string). */
 const char* fa_status_string(int status);
 

@@ -10,6 +10,7 @@
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd2.cuh"
+#include "fa_unfused.cuh"
 
 namespace {
 
@@ -101,6 +102,10 @@ int device_ready(int* sms, int* pair_clusters = nullptr) {
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, true>, fa::DqCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<false>, fa::Fwd2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<true>, fa::Fwd2Cfg::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_unf_scores_kernel<64>, fa::UnfScoresCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_unf_scores_kernel<128>, fa::UnfScoresCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_unf_pv_kernel<64>, fa::UnfPvCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_unf_pv_kernel<128>, fa::UnfPvCfg<128>::SMEM_BYTES);
     for (int c = 0; c < 2 && ok; ++c) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -272,6 +277,70 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   } else {
     if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
     else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+  }
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// standard (unfused) forward: S and P through HBM
+// ---------------------------------------------------------------------------
+static size_t unfused_rows_padded(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+
+size_t fa_fwd_unfused_workspace_bytes(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d)) return 0;
+  const size_t nr = unfused_rows_padded(N);
+  return static_cast<size_t>(B) * H * nr * nr * 2;
+}
+
+int fa_fwd_unfused(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+                   int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, d);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FA_ERR_ALIGNMENT;
+  bool scale_ok = false;
+  const float sc = effective_scale(scale, d, &scale_ok);
+  if (!scale_ok) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_fwd_unfused_workspace_bytes(B, H, N, d);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  const int BH = B * H;
+  const long long nt = static_cast<long long>(unfused_rows_padded(N) / 128);
+  if (static_cast<long long>(BH) * nt * nt > 0x7fffffffLL) return FA_ERR_INVALID_ARG;  // grid limit
+  const size_t tbytes = static_cast<size_t>(BH) * N * d * 2, lbytes = static_cast<size_t>(BH) * N * 4;
+  const Range rq{(uintptr_t)Q, (uintptr_t)Q + tbytes}, rk{(uintptr_t)K, (uintptr_t)K + tbytes},
+      rv{(uintptr_t)V, (uintptr_t)V + tbytes}, ro{(uintptr_t)O, (uintptr_t)O + tbytes},
+      rl{(uintptr_t)LSE, (uintptr_t)LSE + lbytes}, rw{(uintptr_t)workspace, (uintptr_t)workspace + need};
+  const Range ins[3] = {rq, rk, rv};
+  for (int b = 0; b < 3; ++b)
+    if (overlaps(ro, ins[b]) || overlaps(rl, ins[b])) return FA_ERR_INVALID_ARG;
+  if (overlaps(ro, rl)) return FA_ERR_INVALID_ARG;
+  if (overlaps(rw, rq) || overlaps(rw, rk) || overlaps(rw, rv) || overlaps(rw, ro) || overlaps(rw, rl))
+    return FA_ERR_WORKSPACE;
+  int sms = 0;
+  if ((rc = device_ready(&sms))) return rc;
+  if (!is_device_ptr(Q) || !is_device_ptr(K) || !is_device_ptr(V) || !is_device_ptr(O) || !is_device_ptr(LSE) ||
+      !is_device_ptr(workspace))
+    return FA_ERR_UNSUPPORTED_DEVICE;
+  const int Nr = static_cast<int>(nt * 128);
+  CUtensorMap mq, mk, mp, mv;
+  if (!make_map(&mq, Q, BH, N, d, 128) || !make_map(&mk, K, BH, N, d, 128) ||
+      !make_map(&mp, workspace, BH, Nr, Nr, 128) || !make_map(&mv, V, BH, N, d, 64))
+    return encode_failed();
+  clear_stale_error();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* S = static_cast<__half*>(workspace);
+  auto* o = static_cast<__nv_bfloat16*>(O);
+  const unsigned grid_s = static_cast<unsigned>(BH * nt * nt), grid_pv = static_cast<unsigned>(BH * nt);
+  const long long rows = static_cast<long long>(BH) * N;
+  const unsigned grid_sm = static_cast<unsigned>((rows + fa::kUnfSoftmaxRows - 1) / fa::kUnfSoftmaxRows);
+  if (d == 64) {
+    fa::fa_unf_scores_kernel<64><<<grid_s, 128, fa::UnfScoresCfg<64>::SMEM_BYTES, s>>>(mq, mk, S, static_cast<int>(nt), Nr, sc);
+    fa::fa_unf_softmax_kernel<<<grid_sm, 256, 0, s>>>(S, LSE, rows, N, Nr, causal ? 1 : 0);
+    fa::fa_unf_pv_kernel<64><<<grid_pv, 128, fa::UnfPvCfg<64>::SMEM_BYTES, s>>>(mp, mv, o, N, Nr);
+  } else {
+    fa::fa_unf_scores_kernel<128><<<grid_s, 128, fa::UnfScoresCfg<128>::SMEM_BYTES, s>>>(mq, mk, S, static_cast<int>(nt), Nr, sc);
+    fa::fa_unf_softmax_kernel<<<grid_sm, 256, 0, s>>>(S, LSE, rows, N, Nr, causal ? 1 : 0);
+    fa::fa_unf_pv_kernel<128><<<grid_pv, 128, fa::UnfPvCfg<128>::SMEM_BYTES, s>>>(mp, mv, o, N, Nr);
   }
   return launch_status();
 }

@@ -316,6 +316,25 @@ __device__ __forceinline__ void mma_ss_k64(uint32_t d_tmem, uint64_t a0, uint64_
       "l"(a0), "l"(b0), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// K = 64, A K-major (+32 B per K step) and B MN-major (16 rows of 128 bytes =
+// +2048 B per K step), both in shared memory.
+__device__ __forceinline__ void mma_ss_k64_bmn(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 ax, bx;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 ax, %1, 2;\n\tadd.s64 bx, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 4;\n\tadd.s64 bx, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 6;\n\tadd.s64 bx, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // A from tensor memory (K-major, 8 columns of packed bf16 per K step of 16),
 // B MN-major in shared memory (16 rows of 128 bytes = +128 per K step).
 // K = 128 (8 steps).

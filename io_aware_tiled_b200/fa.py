@@ -71,6 +71,10 @@ def load_library(build_if_missing: bool = True):
         lib.fa_last_cuda_error.restype = i
         lib.fa_status_string.argtypes = [i]
         lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_fwd_unfused_workspace_bytes.argtypes = [i, i, i, i]
+        lib.fa_fwd_unfused_workspace_bytes.restype = sz
+        lib.fa_fwd_unfused.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+        lib.fa_fwd_unfused.restype = i
         lib.fa_fwd_kernel_name.argtypes = [i, i]
         lib.fa_fwd_kernel_name.restype = ctypes.c_char_p
         lib.fa_bwd_set_phase_events.argtypes = [vp, vp, vp, vp]
@@ -135,6 +139,30 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
                         int(bool(causal)), _scale(scale, d), _stream_handle(q.device))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
+    return o, l
+
+
+def unfused_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_fwd_unfused_workspace_bytes(B, H, N, d))
+
+
+def forward_unfused(q, k, v, causal: bool = False, scale: float | None = None, workspace=None, out=None,
+                    lse=None):
+    """forward() the standard way: S and P materialised in HBM (fa_fwd_unfused).
+    For measuring the traffic the tiled kernels avoid; same outputs."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    lib = load_library()
+    nbytes = int(lib.fa_fwd_unfused_workspace_bytes(B, H, N, d))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    with torch.cuda.device(q.device):
+        rc = lib.fa_fwd_unfused(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
+                                int(bool(causal)), _scale(scale, d), ws.data_ptr(), ws.numel(),
+                                _stream_handle(q.device))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_unfused")
     return o, l
 
 

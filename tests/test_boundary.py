@@ -24,7 +24,8 @@ def test_every_declared_symbol_is_exported(lib):
     names = fa.header_functions()
     assert set(names) == {"fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_sync_status", "fa_last_error_word",
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
-                          "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name"}
+                          "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name",
+                          "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:
@@ -100,6 +101,37 @@ def test_backward_rejects_bad_arguments(lib):
     assert _bwd(lib, dq=A) == EINVAL              # dQ aliases Q
     assert _bwd(lib, dv=8 * A) == EINVAL          # dV aliases dK
     assert _bwd(lib, ws=9 * A) == EWS             # workspace aliases dV
+
+
+def _unf(lib, ws=20 * A, ws_bytes=None, B=1, H=1, N=128, d=64, causal=0, scale=0.0, **ptrs):
+    p = dict(q=A, k=2 * A, v=3 * A, o=4 * A, lse=5 * A)
+    p.update(ptrs)
+    nb = lib.fa_fwd_unfused_workspace_bytes(B, H, N, d) if ws_bytes is None else ws_bytes
+    return lib.fa_fwd_unfused(p["q"], p["k"], p["v"], p["o"], p["lse"], B, H, N, d, causal, scale, ws, nb, None)
+
+
+def test_unfused_workspace_bytes(lib):
+    # S and then P, 16-bit, [B*H][Nr][Nr] with Nr = N rounded up to 128
+    assert lib.fa_fwd_unfused_workspace_bytes(2, 16, 4096, 128) == 2 * 16 * 4096 * 4096 * 2
+    assert lib.fa_fwd_unfused_workspace_bytes(8, 12, 1000, 64) == 8 * 12 * 1024 * 1024 * 2
+    assert lib.fa_fwd_unfused_workspace_bytes(1, 1, 1, 64) == 128 * 128 * 2
+    assert lib.fa_fwd_unfused_workspace_bytes(1, 1, 0, 64) == 0
+    assert lib.fa_fwd_unfused_workspace_bytes(1, 1, 16, 96) == 0
+
+
+def test_unfused_rejects_bad_arguments(lib):
+    assert _unf(lib, N=0) == EINVAL
+    assert _unf(lib, d=32) == EINVAL
+    assert _unf(lib, q=0) == EINVAL
+    assert _unf(lib, o=4 * A + 2) == EALIGN
+    assert _unf(lib, scale=float("nan")) == EINVAL
+    assert _unf(lib, o=2 * A) == EINVAL            # O aliases K
+    assert _unf(lib, ws=0) == EWS
+    assert _unf(lib, ws=20 * A + 8) == EWS
+    assert _unf(lib, ws_bytes=1024) == EWS
+    assert _unf(lib, ws=3 * A) == EWS              # workspace aliases V
+    if not torch.cuda.is_available():
+        assert _unf(lib) == EDEV
 
 
 def test_selftest_rejects_bad_limit(lib):
