@@ -467,6 +467,75 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+def run_tile_sweep(steps: int, warmup: int):
+    """Forward TFLOP/s of every tile shape the kernels build, B=2, H=16,
+    N=4096, d in {64, 128}, with and without the causal mask, beside the
+    working set each shape needs (the SRAM model of the first page's section
+    1.2, and this layout's shared- and tensor-memory bytes per SM).  One JSON
+    line per point."""
+    import torch
+
+    from io_aware_tiled_b200 import fa
+    from io_aware_tiled_b200.inputs import attention_inputs
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    B, H, N = 2, 16, 4096
+    # (name, FA_FWD_PAIR, FA_FWD_BN, query rows per SM, key tile, stages of K and V, S buffers)
+    forms = [("one-SM", "0", "128", 256, 128, None, 2), ("one-SM", "0", "64", 256, 64, None, 2),
+             ("paired", "1", "128", 128, 128, 5, 3)]
+    for d in (64, 128):
+        q, k, v, _ = (t.to(dev) if t is not None else None
+                      for t in attention_inputs(B, H, N, d, seed=0, with_do=False))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        for name, pair, bn, tq, tk, st, ns in forms:
+            if name == "paired" and d != 128:
+                continue
+            if st is None:
+                st = ((2 if d == 128 else 4) * 128) // tk
+            for causal in (False, True):
+                os.environ["FA_FWD_PAIR"], os.environ["FA_FWD_BN"] = pair, bn
+                try:
+                    kname = fa.forward_kernel_name(d, causal)
+                    for _ in range(warmup):
+                        fa.forward(q, k, v, causal, out=o, lse=lse)
+                    ts = []
+                    for _ in range(steps):
+                        flush.zero_()
+                        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a_.record()
+                        fa.forward(q, k, v, causal, out=o, lse=lse)
+                        b_.record()
+                        torch.cuda.synchronize()
+                        ts.append(a_.elapsed_time(b_))
+                    rc = fa.sync_status(dev)
+                finally:
+                    del os.environ["FA_FWD_PAIR"], os.environ["FA_FWD_BN"]
+                if rc != fa.FA_OK:
+                    raise RuntimeError(f"library status {fa.status_string(rc)}")
+                ms = statistics.median(ts)
+                f, _ = _flops(B, H, N, d, causal)
+                bq = 128  # query rows per softmax warpgroup / TMEM lane block
+                q_tiles_per_sm = tq // bq
+                smem = q_tiles_per_sm * bq * d * 2 + st * 2 * (tk if name == "one-SM" else tk // 2) * d * 2
+                tmem_cols = ns * tk + q_tiles_per_sm * d if name == "one-SM" else ns * tk + d
+                pages_sram = bq * d * 2 + 2 * tk * d * 2 + bq * tk * 2 + bq * d * 2 + bq * 8
+                print(json.dumps({
+                    "sweep": "forward tile shape", "kernel": kname, "form": name, "d": d, "causal": causal,
+                    "T_q_per_sm": tq, "T_k": tk, "kv_stages": st,
+                    "tflops": f / (ms * 1e-3) / 1e12, "ms": ms,
+                    "smem_bytes_per_sm": smem, "tmem_columns": tmem_cols,
+                    "pages_sram_model_bytes": pages_sram,
+                    "config": {"B": B, "H": H, "N": N, "l2": "256 MiB written between timed calls"}}),
+                    flush=True)
+    # shapes that do not fit this layout (not built)
+    print(json.dumps({"sweep": "forward tile shape", "not_built": [
+        "T_k=256 with two 128-row Q tiles per SM: S 2x256 + O 2xd TMEM columns > 512",
+        "T_q=64 per MMA: M=64 tcgen05 tiles use half the TMEM lanes and half the MMA rate",
+        "T_q=256 on one SM: cta_group::1 MMAs stop at M=128; 256 rows per pair is the paired form"]}))
+    return 0
+
+
 def run_ncu_case(case: str, batch: int):
     """A few launches of one kernel family, untimed, for ncu captures: the
     headline shape with B=`batch` (B=4: Q, K, V, O, dO are 67 MB each, so the
@@ -503,7 +572,11 @@ def main(argv=None):
     ap.add_argument("--ncu-case", choices=["fwd", "fwd_causal", "bwd", "bwd_causal", "fwd_unfused"], default=None,
                     help="run a few untimed launches for an ncu capture and exit")
     ap.add_argument("--ncu-batch", type=int, default=4)
+    ap.add_argument("--tile-sweep", action="store_true",
+                    help="time the forward for every tile shape the kernels build and exit")
     args = ap.parse_args(argv)
+    if args.tile_sweep:
+        return run_tile_sweep(max(args.steps, 5), max(args.warmup, 3))
     if args.ncu_case:
         return run_ncu_case(args.ncu_case, args.ncu_batch)
 

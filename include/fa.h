@@ -58,7 +58,12 @@ typedef enum {
  * Forward pass.
  * In:  Q, K, V [B,H,N,d] bf16.
  * Out: O [B,H,N,d] bf16 (O = P V, rounded to nearest even), LSE [B,H,N] fp32.
- * One persistent kernel launch on `stream`.
+ * One persistent kernel launch on `stream`: CTA pairs (fa_fwd_2sm_kernel) for
+ * d = 128 without the mask, one SM per CTA (fa_fwd_kernel) otherwise.  Two
+ * environment variables, read at each call, select other forms for
+ * comparisons: FA_FWD_PAIR=0 / =1 forces the one-SM / paired kernel for
+ * d = 128; FA_FWD_BN=64 runs the one-SM kernel with 64-key K/V tiles instead
+ * of 128.  All forms compute the same O and LSE.
  * Returns FA_OK or an fa_status error code (nothing written on error).
  */
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
@@ -166,8 +171,8 @@ const char* fa_status_string(int status);
 /*
  * Name of the kernel fa_fwd launches on the current device for head size d
  * and the given mask flag: "fa_fwd_2sm_kernel" (CTA pairs, d = 128 without
- * the mask) or "fa_fwd_kernel".  The environment variable FA_FWD_PAIR=0 / =1
- * forces the one or the other for d = 128.  NULL when d is not 64 or 128 or
+ * the mask) or "fa_fwd_kernel", following FA_FWD_PAIR and FA_FWD_BN as
+ * fa_fwd does.  NULL when d is not 64 or 128 or
  * the device is not usable.  Static string, owned by the library.  For
  * labelling timings and profiles; the paper has no counterpart.
  */

@@ -92,6 +92,10 @@ int device_ready(int* sms, int* pair_clusters = nullptr) {
     ok = ok && set_smem(fa::fa_fwd_kernel<64, true>, fa::FwdCfg<64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_kernel<128, false>, fa::FwdCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_kernel<128, true>, fa::FwdCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, false, 64>, fa::FwdCfg<64, 64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, true, 64>, fa::FwdCfg<64, 64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, false, 64>, fa::FwdCfg<128, 64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, true, 64>, fa::FwdCfg<128, 64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<64, false>, fa::DkdvCfg<64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<64, true>, fa::DkdvCfg<64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dkdv_kernel<128, false>, fa::DkdvCfg<128>::SMEM_BYTES);
@@ -211,12 +215,19 @@ const char* fa_status_string(int status) {
 // d = 128 non-causal: the paired (2-SM) kernel (faster there); causal and
 // d = 64 run the 1-SM kernel.  FA_FWD_PAIR=0 / =1 forces one or the other for
 // d = 128 (comparisons and tests).  `clusters`: CTA pairs that fit at once.
+// Keys per K/V tile of the one-SM kernel: 128, or 64 when FA_FWD_BN=64
+// (tile-size comparisons; 64-key tiles also rule out the paired kernel).
+static int fwd_key_tile() {
+  const char* bn_env = getenv("FA_FWD_BN");
+  return (bn_env && strcmp(bn_env, "64") == 0) ? 64 : 128;
+}
+
 static bool fwd_use_pair(int d, int causal, int clusters) {
   const char* pair_env = getenv("FA_FWD_PAIR");
   bool use_pair = d == 128 && clusters > 0 && !causal;
   if (pair_env && strcmp(pair_env, "0") == 0) use_pair = false;
   if (pair_env && strcmp(pair_env, "1") == 0) use_pair = d == 128 && clusters > 0;
-  return use_pair;
+  return use_pair && fwd_key_tile() == 128;
 }
 
 const char* fa_fwd_kernel_name(int d, int causal) {
@@ -271,6 +282,18 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   const float sl2 = sc * fa::kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* o = static_cast<__nv_bfloat16*>(O);
+  if (fwd_key_tile() == 64) {  // 64-key tiles: for tile-size comparisons only
+    CUtensorMap mk64, mv64;
+    if (!make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64)) return encode_failed();
+    if (d == 64) {
+      if (causal) fa::fa_fwd_kernel<64, true, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
+      else fa::fa_fwd_kernel<64, false, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
+    } else {
+      if (causal) fa::fa_fwd_kernel<128, true, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
+      else fa::fa_fwd_kernel<128, false, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
+    }
+    return launch_status();
+  }
   if (d == 64) {
     if (causal) fa::fa_fwd_kernel<64, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
     else fa::fa_fwd_kernel<64, false><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);

@@ -37,15 +37,17 @@
 
 namespace fa {
 
-template <int D>
+template <int D, int BN_ = 128>
 struct FwdCfg {
   static constexpr int BM = 128;                 // query rows per Q tile
-  static constexpr int BN = 128;                 // keys per K/V tile
+  static constexpr int BN = BN_;                 // keys per K/V tile: 128, or 64 (tile-size comparisons)
+  static constexpr int R = BM / BN;              // key tiles per query tile's width
   static constexpr int CH = D / 64;              // 128-byte column chunks per row
-  static constexpr int CHUNK = 128 * 128;        // bytes of one 64-column chunk of a 128-row tile
+  static constexpr int CHUNK = 128 * 128;        // bytes of one 64-column chunk of a 128-row Q tile
+  static constexpr int KV_CHUNK = BN * 128;      // bytes of one 64-column chunk of a K or V tile
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int KV_TILE = BN * D * 2;
-  static constexpr int ST = (D == 128) ? 2 : 4;  // K and V ring depth
+  static constexpr int ST = ((D == 128) ? 2 : 4) * R;  // K and V ring depth (same bytes for either BN)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + ST * KV_TILE;
@@ -58,7 +60,7 @@ struct FwdCfg {
   static constexpr int NUM_BARS = B_O_EMPTY + 2;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;  // + room to align the base to 1024
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = BN, TM_O0 = 256, TM_O1 = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
   // warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 idle; warpgroups 1 and 2: softmax of Q tile 0 and 1
   static constexpr int THREADS = 384;
@@ -87,12 +89,12 @@ __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool caus
   }
 }
 
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+template <int D, bool CAUSAL, int BN_ = 128>
+__global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
                   float* __restrict__ LSE, int BH, int N, float scale_log2) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, BN_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       for (int k = 0, u = blockIdx.x; u < units; u = serpentine_unit(++k, blockIdx.x, gridDim.x)) {
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
-        const int nk1 = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
+        const int nk1 = CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT;
         if (!mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it & 1) ^ 1, FW_PROD_Q)) break;
         ++q_it;
         mbar_arrive_expect_tx(bars + 8 * C::B_Q_FULL, 2 * C::Q_TILE);
@@ -163,12 +165,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           if (!mbar_wait(bars + 8 * (C::B_K_EMPTY + s), ph ^ 1, FW_PROD_K)) { ok = false; break; }
           mbar_arrive_expect_tx(bars + 8 * (C::B_K_FULL + s), C::KV_TILE);
           for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(sK + s * C::KV_TILE + c * C::CHUNK, &tmK, bars + 8 * (C::B_K_FULL + s), c * 64,
+            tma_load_3d(sK + s * C::KV_TILE + c * C::KV_CHUNK, &tmK, bars + 8 * (C::B_K_FULL + s), c * 64,
                         j * C::BN, bh);
           if (!mbar_wait(bars + 8 * (C::B_V_EMPTY + s), ph ^ 1, FW_PROD_V)) { ok = false; break; }
           mbar_arrive_expect_tx(bars + 8 * (C::B_V_FULL + s), C::KV_TILE);
           for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(sV + s * C::KV_TILE + c * C::CHUNK, &tmV, bars + 8 * (C::B_V_FULL + s), c * 64,
+            tma_load_3d(sV + s * C::KV_TILE + c * C::KV_CHUNK, &tmV, bars + 8 * (C::B_V_FULL + s), c * 64,
                         j * C::BN, bh);
         }
         if (!ok) break;
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     // The whole warp runs this loop with warp-uniform values; one elected lane
     // issues each tcgen05.mma / commit.
     {
-      constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t IDESC_S = idesc_bf16(128, C::BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
       // S = Q_t K_j^T: K = d in steps of 16 (one 8- or 4-MMA group).
       auto issue_s = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
@@ -187,14 +189,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const uint64_t a0 = sdesc_make(sdesc_lo(a_smem, 16), hi), b0 = sdesc_make(sdesc_lo(b_smem, 16), hi);
         if (D == 128)
           mma_ss_k128(d_tmem, a0, sdesc_make(sdesc_lo(a_smem + C::CHUNK, 16), hi), b0,
-                      sdesc_make(sdesc_lo(b_smem + C::CHUNK, 16), hi), IDESC_S, 0u);
+                      sdesc_make(sdesc_lo(b_smem + C::KV_CHUNK, 16), hi), IDESC_S, 0u);
         else
           mma_ss_k64(d_tmem, a0, b0, IDESC_S, 0u);
       };
-      // O_t += P_t V_j: 8 steps of 16 keys; P_t from tensor memory, V_j MN-major.
+      // O_t += P_t V_j: BN/16 steps of 16 keys; P_t from tensor memory, V_j MN-major.
       auto issue_pv = [&](uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, bool acc) {
-        mma_ts_k128(d_tmem, p_tmem, sdesc_make(sdesc_lo(v_smem, C::CHUNK), sdesc_hi(1024)), IDESC_PV,
-                    acc ? 1u : 0u);
+        const uint64_t vd = sdesc_make(sdesc_lo(v_smem, C::KV_CHUNK), sdesc_hi(1024));
+        if (C::BN == 128)
+          mma_ts_k128(d_tmem, p_tmem, vd, IDESC_PV, acc ? 1u : 0u);
+        else
+          mma_ts_k64(d_tmem, p_tmem, vd, IDESC_PV, acc ? 1u : 0u);
       };
       uint32_t kv_it = 0, q_it = 0, unit_it = 0;
       uint32_t p_ph0 = 0, p_ph1 = 0;
@@ -202,8 +207,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
         (void)bh;
-        const int nk0 = CAUSAL ? min(2 * qp + 1, NKT) : NKT;
-        const int nk1 = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
+        const int nk0 = CAUSAL ? min((2 * qp + 1) * C::R, NKT) : NKT;
+        const int nk1 = CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT;
         bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_FULL, q_it & 1, FW_MMA_Q));
         ++q_it;
         if (!ok) break;
@@ -288,26 +293,30 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       int bh, qp;
       fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
       const int qt = 2 * qp + wg;
-      const int nk = CAUSAL ? min(qt + 1, NKT) : NKT;
+      const int nk = CAUSAL ? min((qt + 1) * C::R, NKT) : NKT;
       const int row = qt * C::BM + r;
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < nk; ++j) {
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s, s_it & 1, FW_SM_S)))) break;
         ++s_it;
         tc_fence_after();
-        uint32_t sr[128];
+        constexpr int NC = C::BN;  // score columns per row
+        uint32_t sr[NC];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        for (int c = 0; c < NC / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-        float s[128];
+        for (int c = 0; c < NC / 32; ++c) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        float s[NC];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        for (int c = 0; c < NC; ++c) s[c] = __uint_as_float(sr[c]);
         const int kbase = j * C::BN;
-        if ((CAUSAL && j == qt) || kbase + C::BN > N) {
+        // the diagonal tiles: some key of the tile lies past some row of the Q tile
+        // (with 128-key tiles exactly the tile j == qt)
+        const bool diag = C::BN == C::BM ? j == qt : kbase + C::BN - 1 > qt * C::BM;
+        if ((CAUSAL && diag) || kbase + C::BN > N) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
+          for (int c = 0; c < NC; ++c) {
             const int key = kbase + c;
             if (key >= N || (CAUSAL && key > row)) s[c] = -INFINITY;
           }
@@ -317,7 +326,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) pm[e] = s[e];
 #pragma unroll
-        for (int c = 8; c < 128; c += 8)
+        for (int c = 8; c < NC; c += 8)
 #pragma unroll
           for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
 #pragma unroll
@@ -336,7 +345,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const float neg = -m_ref;
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {  // 32 scores -> 16 packed bf16 pairs -> 16 TMEM columns
+        for (int ch = 0; ch < NC / 32; ++ch) {  // 32 scores -> 16 packed bf16 pairs -> 16 TMEM columns
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {

@@ -354,3 +354,24 @@ def test_forward_kernel_name_follows_the_routing(monkeypatch):
     assert fa.forward_kernel_name(64, True) == "fa_fwd_kernel"
     with pytest.raises(RuntimeError):
         fa.forward_kernel_name(96, False)
+
+
+BN64_CASES = [(1, 2, 1000, 128, True), (1, 2, 1000, 128, False), (1, 1, 129, 64, True), (2, 2, 300, 64, False),
+              (1, 1, 1, 128, True), (1, 3, 640, 128, True), (1, 1, 200, 64, True)]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", BN64_CASES)
+def test_forward_with_64_key_tiles(B, H, N, d, causal, monkeypatch):
+    """FA_FWD_BN=64 runs the one-SM kernel with 64-key K/V tiles (tile-size
+    comparisons): two key tiles per query tile's width, so the causal
+    diagonal spans two tiles and the second may be fully masked for half the
+    rows."""
+    q, k, v, _ = attention_inputs(B, H, N, d, seed=31 + N + d, with_do=False)
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), causal, 1 / d ** 0.5)
+    monkeypatch.setenv("FA_FWD_BN", "64")
+    assert fa.forward_kernel_name(d, causal) == "fa_fwd_kernel"
+    o, lse = _run_fwd(q, k, v, causal)
+    monkeypatch.delenv("FA_FWD_BN")
+    what = f"64-key tiles {B,H,N,d} causal={causal}"
+    check_o(f64(o), ro, what)
+    check_lse(f64(lse), rl, what)
