@@ -467,6 +467,71 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+def run_all_configs(steps: int, warmup: int):
+    """Every named workload on one GPU: forward (each mask it names) and, where
+    it names one, forward + backward; CUDA events around each call, the L2
+    flushed before each (the small single-head workload also without the
+    flush), median and best of `steps` calls after `warmup`.  One JSON line
+    per (workload, mask, pass)."""
+    import torch
+
+    from io_aware_tiled_b200 import fa
+    from io_aware_tiled_b200.configs import WORKLOADS
+    from io_aware_tiled_b200.inputs import attention_inputs
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peak = _peaks()["bf16_tflops"]
+
+    def time_calls(fn, do_flush):
+        for _ in range(warmup):
+            fn()
+        ts = []
+        for _ in range(steps):
+            if do_flush:
+                flush.zero_()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record()
+            fn()
+            b_.record()
+            torch.cuda.synchronize()
+            ts.append(a_.elapsed_time(b_))
+        rc = fa.sync_status(dev)
+        if rc != fa.FA_OK:
+            raise RuntimeError(f"library status {fa.status_string(rc)}")
+        return statistics.median(ts), min(ts)
+
+    for w in WORKLOADS.values():
+        q, k, v, do = (t.to(dev) for t in attention_inputs(w.B, w.H, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        ws = torch.empty(fa.workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        io_bytes = w.B * w.H * w.N * (4 * w.d * 2 + 4)  # Q, K, V read; O written; LSE written
+        for causal in w.causal_modes:
+            passes = [("fwd", lambda: fa.forward(q, k, v, causal, out=o, lse=lse), w.fwd_flops(causal))]
+            if w.backward:
+                passes.append(("fwd+bwd", lambda: (fa.forward(q, k, v, causal, out=o, lse=lse),
+                                                   fa.backward(q, k, v, o, do, lse, causal, workspace=ws,
+                                                               dq=dq, dk=dk, dv=dv)),
+                               w.fwd_flops(causal) + w.bwd_flops(causal)))
+            for name, fn, flops in passes:
+                for do_flush in ((True, False) if w.N * w.B * w.H <= 4096 else (True,)):
+                    med, best = time_calls(fn, do_flush)
+                    line = {"workload": w.name, "causal": causal, "pass": name,
+                            "kernel": fa.forward_kernel_name(w.d, causal),
+                            "median_us": med * 1e3, "best_us": best * 1e3,
+                            "tflops_median": flops / (med * 1e-3) / 1e12, "tflops_best": flops / (best * 1e-3) / 1e12,
+                            "frac_of_measured_peak_median": flops / (med * 1e-3) / 1e12 / peak,
+                            "l2": "flushed before each call" if do_flush else "warm (no flush)",
+                            "steps": steps, "warmup": warmup}
+                    if name == "fwd":
+                        line["gbs_median"] = io_bytes / (med * 1e-3) / 1e9
+                    print(json.dumps(line), flush=True)
+        del q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+    return 0
+
+
 def run_tile_sweep(steps: int, warmup: int):
     """Forward TFLOP/s of every tile shape the kernels build, B=2, H=16,
     N=4096, d in {64, 128}, with and without the causal mask, beside the
@@ -528,6 +593,37 @@ def run_tile_sweep(steps: int, warmup: int):
                     "pages_sram_model_bytes": pages_sram,
                     "config": {"B": B, "H": H, "N": N, "l2": "256 MiB written between timed calls"}}),
                     flush=True)
+    # the online-softmax rescale threshold (default kernels)
+    for d in (64, 128):
+        q, k, v, _ = (t.to(dev) if t is not None else None
+                      for t in attention_inputs(B, H, N, d, seed=0, with_do=False))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        for causal in (False, True):
+            for thr in ("0", "8", "16"):
+                os.environ["FA_FWD_RESCALE"] = thr
+                try:
+                    for _ in range(warmup):
+                        fa.forward(q, k, v, causal, out=o, lse=lse)
+                    ts = []
+                    for _ in range(steps):
+                        flush.zero_()
+                        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a_.record()
+                        fa.forward(q, k, v, causal, out=o, lse=lse)
+                        b_.record()
+                        torch.cuda.synchronize()
+                        ts.append(a_.elapsed_time(b_))
+                    rc = fa.sync_status(dev)
+                finally:
+                    del os.environ["FA_FWD_RESCALE"]
+                if rc != fa.FA_OK:
+                    raise RuntimeError(f"library status {fa.status_string(rc)}")
+                ms = statistics.median(ts)
+                f, _ = _flops(B, H, N, d, causal)
+                print(json.dumps({"sweep": "rescale threshold (log2)", "threshold": float(thr),
+                                  "kernel": fa.forward_kernel_name(d, causal), "d": d, "causal": causal,
+                                  "tflops": f / (ms * 1e-3) / 1e12, "ms": ms}), flush=True)
     # shapes that do not fit this layout (not built)
     print(json.dumps({"sweep": "forward tile shape", "not_built": [
         "T_k=256 with two 128-row Q tiles per SM: S 2x256 + O 2xd TMEM columns > 512",
@@ -574,7 +670,11 @@ def main(argv=None):
     ap.add_argument("--ncu-batch", type=int, default=4)
     ap.add_argument("--tile-sweep", action="store_true",
                     help="time the forward for every tile shape the kernels build and exit")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="time every named workload (fwd, fwd+bwd) and exit")
     args = ap.parse_args(argv)
+    if args.all_configs:
+        return run_all_configs(max(args.steps, 50), max(args.warmup, 10))
     if args.tile_sweep:
         return run_tile_sweep(max(args.steps, 5), max(args.warmup, 3))
     if args.ncu_case:

@@ -63,7 +63,9 @@ typedef enum {
  * environment variables, read at each call, select other forms for
  * comparisons: FA_FWD_PAIR=0 / =1 forces the one-SM / paired kernel for
  * d = 128; FA_FWD_BN=64 runs the one-SM kernel with 64-key K/V tiles instead
- * of 128.  All forms compute the same O and LSE.
+ * of 128.  FA_FWD_RESCALE=t (0 .. 30, default 8) sets the online-softmax
+ * rescale threshold: O is rescaled only when a row maximum grows by more than
+ * a factor 2^t.  All forms compute the same O and LSE up to rounding.
  * Returns FA_OK or an fa_status error code (nothing written on error).
  */
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,

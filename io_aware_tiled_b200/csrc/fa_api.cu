@@ -222,6 +222,18 @@ static int fwd_key_tile() {
   return (bn_env && strcmp(bn_env, "64") == 0) ? 64 : 128;
 }
 
+// Online-softmax rescale threshold in log2 units: O is rescaled only when a
+// row max grows by more than 2^threshold.  FA_FWD_RESCALE (0 .. 30) overrides
+// the default 8; 0 rescales on every growth.  Any value gives the same result
+// up to rounding: P stays below 2^threshold, far inside fp32 and bf16 range.
+static float fwd_rescale_log2() {
+  const char* env = getenv("FA_FWD_RESCALE");
+  if (!env) return 8.f;
+  char* end = nullptr;
+  const float v = strtof(env, &end);
+  return (end != env && v >= 0.f && v <= 30.f) ? v : 8.f;
+}
+
 static bool fwd_use_pair(int d, int causal, int clusters) {
   const char* pair_env = getenv("FA_FWD_PAIR");
   bool use_pair = d == 128 && clusters > 0 && !causal;
@@ -262,6 +274,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   if (!make_map(&mq, Q, BH, N, d, 128) || !make_map(&mk, K, BH, N, d, 128) || !make_map(&mv, V, BH, N, d, 128))
     return encode_failed();
   clear_stale_error();
+  const float rescale = fwd_rescale_log2();
   const int clusters = pair_clusters[causal ? 1 : 0];
   if (fwd_use_pair(d, causal, clusters)) {
     CUtensorMap mkh;
@@ -272,9 +285,9 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
     cudaStream_t sp = static_cast<cudaStream_t>(stream);
     auto* op = static_cast<__nv_bfloat16*>(O);
     if (causal)
-      fa::fa_fwd_2sm_kernel<true><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p);
+      fa::fa_fwd_2sm_kernel<true><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p, rescale);
     else
-      fa::fa_fwd_2sm_kernel<false><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p);
+      fa::fa_fwd_2sm_kernel<false><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p, rescale);
     return launch_status();
   }
   const int nqt = (N + 127) / 128, units = BH * ((nqt + 1) / 2);
@@ -286,20 +299,20 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
     CUtensorMap mk64, mv64;
     if (!make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64)) return encode_failed();
     if (d == 64) {
-      if (causal) fa::fa_fwd_kernel<64, true, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
-      else fa::fa_fwd_kernel<64, false, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
+      if (causal) fa::fa_fwd_kernel<64, true, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
+      else fa::fa_fwd_kernel<64, false, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
     } else {
-      if (causal) fa::fa_fwd_kernel<128, true, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
-      else fa::fa_fwd_kernel<128, false, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2);
+      if (causal) fa::fa_fwd_kernel<128, true, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
+      else fa::fa_fwd_kernel<128, false, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
     }
     return launch_status();
   }
   if (d == 64) {
-    if (causal) fa::fa_fwd_kernel<64, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
-    else fa::fa_fwd_kernel<64, false><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+    if (causal) fa::fa_fwd_kernel<64, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
+    else fa::fa_fwd_kernel<64, false><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
   } else {
-    if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
-    else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2);
+    if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
+    else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
   }
   return launch_status();
 }

@@ -553,6 +553,26 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^t on the FMA and integer pipes instead of the MUFU, for t <= 8 (the
+// softmax arguments; -inf included).  Cody-Waite range reduction: 2^t =
+// 2^j 2^f with j = rint(t) (added 1.5 * 2^23 leaves j in the low mantissa
+// bits of r) and f = t - j in [-1/2, 1/2]; 2^f from the degree-3 polynomial of
+// least maximum relative error on that interval (Remez exchange, fitted by
+// fit_exp2_poly.py); j is added to the exponent field.  Relative error
+// <= 7.5e-5 on [-125, 8], below bf16's rounding of P (2^-9).  t is clamped at
+// -126 so the exponent field never wraps: smaller arguments (masked scores
+// are -inf) give a positive value <= 2^-125 (not 0), which no fp32 sum or
+// bf16 product can register.
+// The softmax sends a fixed share of its exponentials here so that the MUFU
+// and the FMA pipes finish together.
+__device__ __forceinline__ float exp2_poly3(float t) {
+  t = fmaxf(t, -126.f);
+  const float r = t + 12582912.f;
+  const float f = t - (r - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.05517166853f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
   return *reinterpret_cast<uint32_t*>(&v);

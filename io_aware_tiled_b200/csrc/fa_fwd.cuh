@@ -29,7 +29,9 @@
 //   * Softmax: each thread owns one full row of S (tcgen05.ld 32x32b), so the
 //     row max and row sum are register reductions.  Work is in base 2 with
 //     scale*log2(e) folded into one FMA.  O is rescaled only when a row's max
-//     grows by more than 2^8 (exact: the final division uses the same max).
+//     grows by more than a factor 2^rescale_log2 (8 by default; exact: the
+//     final division uses the same max).  A fixed share of the exponentials
+//     runs on the FMA pipe (exp2_poly3), the rest on the MUFU.
 //   * Epilogue: O / l as bf16 and LSE as fp32, stored once per row.
 #pragma once
 
@@ -66,7 +68,9 @@ struct FwdCfg {
   static constexpr int THREADS = 384;
   // register split (launch: 384 threads x 168): control warpgroup 56, softmax warpgroups 216 each
   static constexpr uint32_t REGS_CONTROL = 56, REGS_SOFTMAX = 216;
-  static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+  // one exponential pair in EXP_EMUL_EVERY goes to exp2_poly3 (FMA pipe)
+  // instead of the MUFU: 1/4 of them at d = 64, 1/8 at d = 128 (measured best)
+  static constexpr int EXP_EMUL_EVERY = (D == 64) ? 4 : 8;
 };
 
 // wait-site identifiers recorded in the error word
@@ -93,7 +97,8 @@ template <int D, bool CAUSAL, int BN_ = 128>
 __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-                  float* __restrict__ LSE, int BH, int N, float scale_log2) {
+                  float* __restrict__ LSE, int BH, int N, float scale_log2,
+                  float rescale_log2) {
   using C = FwdCfg<D, BN_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -335,7 +340,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
         const float mx = pm[0];
         const float m_new = fmaxf(m_ref, mx * scale_log2);
-        const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
+        const bool need = m_new > m_ref + rescale_log2;
         const bool warp_rescale = __any_sync(0xffffffffu, need);
         const float alpha = need ? ex2(m_ref - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
         if (need) {
@@ -349,8 +354,11 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(s[32 * ch + 2 * c], scale_log2, neg));
-            const float p1 = ex2(fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg));
+            const float t0 = fmaf(s[32 * ch + 2 * c], scale_log2, neg);
+            const float t1 = fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg);
+            const bool emul = c % C::EXP_EMUL_EVERY == C::EXP_EMUL_EVERY - 1;  // resolved at compile time
+            const float p0 = emul ? exp2_poly3(t0) : ex2(t0);
+            const float p1 = emul ? exp2_poly3(t1) : ex2(t1);
             ps[c & 7] += p0 + p1;
             p[c] = pack_bf16(p0, p1);
           }

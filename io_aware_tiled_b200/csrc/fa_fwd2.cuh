@@ -25,8 +25,10 @@
 //   * Softmax: two warpgroups per CTA split every row's 128 scores (64 each);
 //     they exchange partial row maxima through shared memory once per step and
 //     combine row sums only at the end.  Base 2; O (each warpgroup its half of
-//     the columns) is rescaled only when a row max grows by more than 2^8, after
-//     waiting for the previous PV (an "O done" barrier committed after every PV).
+//     the columns) is rescaled only when a row max grows by more than a factor
+//     2^rescale_log2 (8 by default), after waiting for the previous PV (an "O
+//     done" barrier committed after every PV).  One exponential in 8 runs on
+//     the FMA pipe (exp2_poly3).
 #pragma once
 
 #include "fa_device.cuh"
@@ -61,7 +63,7 @@ struct Fwd2Cfg {
   // warp 0 loads, warp 1 MMA (leader) or relay (peer), warps 4-7 and 8-11: the
   // softmax warpgroups of the low and the high 64 columns
   static constexpr int THREADS = 384;
-  static constexpr float RESCALE_THRESHOLD = 8.0f;
+  static constexpr int EXP_EMUL_EVERY = 8;  // 1/8 of the exponentials on the FMA pipe (exp2_poly3)
   static constexpr uint16_t BOTH = 0x3;          // multicast mask: both CTAs of the pair
 };
 
@@ -87,7 +89,8 @@ template <bool CAUSAL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     fa_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKh,
                       const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-                      float* __restrict__ LSE, int BH, int N, float scale_log2) {
+                      float* __restrict__ LSE, int BH, int N, float scale_log2,
+                  float rescale_log2) {
   using C = Fwd2Cfg;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -327,7 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
         // Both halves have loaded their S before that barrier, so from here on
         // P may be written over S's columns.
         const float m_new = fmaxf(m_ref, mx * scale_log2);
-        const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
+        const bool need = m_new > m_ref + rescale_log2;
         const bool warp_rescale = __any_sync(0xffffffffu, need);
         const float alpha = need ? ex2(m_ref - m_new) : 1.f;  // ex2(-inf) = 0 on the first tile
         if (need) {
@@ -342,8 +345,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(s[32 * ch + 2 * c], scale_log2, neg));
-            const float p1 = ex2(fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg));
+            const float t0 = fmaf(s[32 * ch + 2 * c], scale_log2, neg);
+            const float t1 = fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg);
+            const bool emul = c % C::EXP_EMUL_EVERY == C::EXP_EMUL_EVERY - 1;  // resolved at compile time
+            const float p0 = emul ? exp2_poly3(t0) : ex2(t0);
+            const float p1 = emul ? exp2_poly3(t1) : ex2(t1);
             ps[c & 7] += p0 + p1;
             p[c] = pack_bf16(p0, p1);
           }

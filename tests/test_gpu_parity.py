@@ -375,3 +375,23 @@ def test_forward_with_64_key_tiles(B, H, N, d, causal, monkeypatch):
     what = f"64-key tiles {B,H,N,d} causal={causal}"
     check_o(f64(o), ro, what)
     check_lse(f64(lse), rl, what)
+
+
+@pytest.mark.parametrize("threshold", ["0", "3", "16", "30"])
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_forward_rescale_threshold(threshold, pair, monkeypatch):
+    """FA_FWD_RESCALE sets how far a row maximum may grow before O is
+    rescaled (0: on every growth).  Logits in the hundreds (sigma 8) make the
+    maxima jump across tiles, so rescaling happens often; every threshold
+    gives the oracle's O and LSE."""
+    B, H, N, d = 1, 2, 777, 128
+    q, k, v, _ = attention_inputs(B, H, N, d, seed=41, sigma_qk=8.0, with_do=False)
+    ro, rl = oracle.forward(f64(q), f64(k), f64(v), True, 1 / d ** 0.5)
+    ro2, rl2 = oracle.forward(f64(q), f64(k), f64(v), False, 1 / d ** 0.5)
+    monkeypatch.setenv("FA_FWD_RESCALE", threshold)
+    monkeypatch.setenv("FA_FWD_PAIR", pair)
+    for causal, (o_ref, l_ref) in ((True, (ro, rl)), (False, (ro2, rl2))):
+        o, lse = _run_fwd(q, k, v, causal)
+        what = f"rescale threshold {threshold} pair={pair} causal={causal}"
+        check_o(f64(o), o_ref, what)
+        check_lse(f64(lse), l_ref, what)
