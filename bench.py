@@ -394,10 +394,20 @@ def run_ours(args, rank, world, local_rank):
         for h, t in zip((ho, hl, hdq, hdk, hdv), (o2, l2, *g)):
             h.copy_(t, non_blocking=True)
 
+    from io_aware_tiled_b200.host_pipeline import forward_backward_host
+
+    def e2e_pipelined():
+        # heads in groups through three streams: copies in, kernels, copies out
+        forward_backward_host(hq, hk, hv, hdo, False, out=(ho, hl, hdq, hdk, hdv), device=dev)
+
+    e2e_steps = max(3, args.steps // 4)
     for _ in range(2):
         e2e_step()
-    e2e_ms, _ = timed(e2e_step, max(3, args.steps // 4))
-    e2e_steps = max(3, args.steps // 4)
+    e2e_serial_ms, _ = timed(e2e_step, e2e_steps)
+    e2e_serial_ms = max_over_ranks(e2e_serial_ms, world, dev)
+    for _ in range(2):
+        e2e_pipelined()
+    e2e_ms, _ = timed(e2e_pipelined, e2e_steps)
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
     d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
@@ -458,8 +468,14 @@ def run_ours(args, rank, world, local_rank):
             },
             "kernels": kernels,
             "roofline": roof,
+            # through forward_backward_host (pinned host in, pinned host out, the
+            # PCIe copies overlapped with the kernels); "serial" copies all
+            # inputs, runs the kernels, then copies all outputs back
             "e2e": {"value": world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps,
+                    "api": "io_aware_tiled_b200.host_pipeline.forward_backward_host",
+                    "serial_value": world * step_flops * e2e_steps / (e2e_serial_ms * 1e-3) / 1e12,
+                    "serial_ms_per_step": e2e_serial_ms / e2e_steps},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
             "peaks": peaks,
@@ -527,6 +543,23 @@ def run_all_configs(steps: int, warmup: int):
                     if name == "fwd":
                         line["gbs_median"] = io_bytes / (med * 1e-3) / 1e9
                     print(json.dumps(line), flush=True)
+                if w.B * w.H * w.N <= 4096:
+                    # latency-bound: the same call replayed from a CUDA graph
+                    # (no host-side work between the events)
+                    fn()
+                    torch.cuda.synchronize()
+                    graph = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+                        fn()
+                    for do_flush in (True, False):
+                        med, best = time_calls(graph.replay, do_flush)
+                        print(json.dumps({"workload": w.name, "causal": causal, "pass": name, "launch": "graph replay",
+                                          "median_us": med * 1e3, "best_us": best * 1e3,
+                                          "tflops_median": flops / (med * 1e-3) / 1e12,
+                                          "gbs_median": io_bytes / (med * 1e-3) / 1e9 if name == "fwd" else None,
+                                          "l2": "flushed before each call" if do_flush else "warm (no flush)",
+                                          "steps": steps, "warmup": warmup}), flush=True)
+                    del graph
         del q, k, v, do, o, lse, dq, dk, dv, ws
         torch.cuda.empty_cache()
     return 0

@@ -395,3 +395,23 @@ def test_forward_rescale_threshold(threshold, pair, monkeypatch):
         what = f"rescale threshold {threshold} pair={pair} causal={causal}"
         check_o(f64(o), o_ref, what)
         check_lse(f64(lse), l_ref, what)
+
+
+def test_host_pipeline_equals_the_device_path():
+    """forward_backward_host (pinned host tensors, heads in groups through
+    three streams) returns exactly the device path's outputs: the same
+    kernels on the same heads, only the copies are scheduled differently."""
+    from io_aware_tiled_b200.host_pipeline import forward_backward_host
+    dev = _dev()
+    B, H, N, d = 2, 3, 300, 128
+    q, k, v, do = attention_inputs(B, H, N, d, seed=77)
+    for causal in (False, True):
+        o, lse = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal)
+        g = fa.backward(q.to(dev), k.to(dev), v.to(dev), o, do.to(dev), lse, causal)
+        host = forward_backward_host(*(t.pin_memory() for t in (q, k, v, do)), causal, groups=4, device=dev)
+        torch.cuda.synchronize()
+        assert fa.sync_status() == fa.FA_OK
+        for got, want in zip(host, (o, lse, *g)):
+            assert torch.equal(got, want.cpu())
+    with pytest.raises(ValueError):
+        forward_backward_host(q, k, v, do)  # not pinned
