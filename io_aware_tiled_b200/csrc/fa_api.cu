@@ -8,6 +8,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd2.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd2.cuh"
 #include "fa_unfused.cuh"
@@ -106,6 +107,8 @@ int device_ready(int* sms, int* pair_clusters = nullptr) {
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, true>, fa::DqCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<false>, fa::Fwd2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<true>, fa::Fwd2Cfg::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_2sm_kernel<false>, fa::Dkdv2Cfg::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_2sm_kernel<true>, fa::Dkdv2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_scores_kernel<64>, fa::UnfScoresCfg<64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_scores_kernel<128>, fa::UnfScoresCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_pv_kernel<64>, fa::UnfPvCfg<64>::SMEM_BYTES);
@@ -447,6 +450,16 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   };
   const int grid_kv = BH * ((N + 127) / 128);
   const int grid_q = BH * ((N + 127) / 128);
+  // FA_BWD_PAIR=1 runs dK/dV on CTA pairs (256 keys per pair, d = 128) for
+  // comparisons: correct, but slower than one SM per 128 keys, because with
+  // two S^T/dP^T buffers (tensor memory is full) each tile waits on two
+  // cross-SM signals.
+  const char* bwd_pair_env = getenv("FA_BWD_PAIR");
+  const bool bwd_pair = d == 128 && bwd_pair_env && strcmp(bwd_pair_env, "1") == 0;
+  CUtensorMap mq32, mdo32;
+  if (bwd_pair && (!make_map(&mq32, Q, BH, N, d, 32) || !make_map(&mdo32, dO, BH, N, d, 32)))
+    return encode_failed();
+  const int grid_kv2 = 2 * BH * ((N + 255) / 256);
   if (d == 64) {
     const long long threads = rows * 8;
     mark(0);
@@ -469,12 +482,18 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
     fa::fa_bwd_preprocess_kernel<128><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(o, dob, Dvec, rows);
     mark(1);
     if (causal) {
-      fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      if (bwd_pair)
+        fa::fa_bwd_dkdv_2sm_kernel<true><<<grid_kv2, fa::Dkdv2Cfg::THREADS, fa::Dkdv2Cfg::SMEM_BYTES, s>>>(mq32, mdo32, mq64, mdo64, mk128, mv128, LSE, Dvec, dk, dv, N, sc, sl2);
+      else
+        fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
       mark(2);
       fa::fa_bwd_dq_kernel<128, true><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
       mark(3);
     } else {
-      fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      if (bwd_pair)
+        fa::fa_bwd_dkdv_2sm_kernel<false><<<grid_kv2, fa::Dkdv2Cfg::THREADS, fa::Dkdv2Cfg::SMEM_BYTES, s>>>(mq32, mdo32, mq64, mdo64, mk128, mv128, LSE, Dvec, dk, dv, N, sc, sl2);
+      else
+        fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
       mark(2);
       fa::fa_bwd_dq_kernel<128, false><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
       mark(3);

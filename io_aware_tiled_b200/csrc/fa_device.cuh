@@ -429,6 +429,25 @@ __device__ __forceinline__ void mma2_ss_k128(uint32_t d_tmem, uint64_t a0, uint6
       "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// K = 64 (4 steps): A from each CTA's tensor memory, B MN-major in each CTA's
+// shared memory (+2048 B per step of 16 rows).
+__device__ __forceinline__ void mma2_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 bx;\n\t.reg .b32 ax;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 ax, %1, 8;\n\tadd.s64 bx, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 16;\n\tadd.s64 bx, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t"
+      "add.s32 ax, %1, 24;\n\tadd.s64 bx, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [ax], bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma2_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(

@@ -415,3 +415,33 @@ def test_host_pipeline_equals_the_device_path():
             assert torch.equal(got, want.cpu())
     with pytest.raises(ValueError):
         forward_backward_host(q, k, v, do)  # not pinned
+
+
+BWD_PAIR_CASES = [(1, 2, 1000, True), (1, 2, 1000, False), (2, 2, 300, True), (1, 1, 200, False),
+                  (1, 1, 1, True), (1, 3, 640, True), (1, 1, 513, False), (1, 2, 129, True)]
+
+
+@pytest.mark.parametrize("B,H,N,causal", BWD_PAIR_CASES)
+def test_both_dkdv_kernels_for_d128(B, H, N, causal, monkeypatch):
+    """d = 128 has two dK/dV kernels: one SM per 128 keys (the default), and
+    CTA pairs per 256 keys (2-SM MMAs, query rows and columns split between
+    the CTAs; FA_BWD_PAIR=1).  Both match the oracle, including N below 256
+    (the second CTA's keys all lie past N) and N = 1."""
+    dev = _dev()
+    d = 128
+    q, k, v, do = attention_inputs(B, H, N, d, seed=5 * N + 3)
+    ref = oracle.backward(f64(q), f64(k), f64(v), f64(do), causal, 1 / d ** 0.5)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = fa.forward(qd, kd, vd, causal)
+    grads = {}
+    for mode in ("0", "1"):
+        monkeypatch.setenv("FA_BWD_PAIR", mode)
+        dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, causal)
+        assert fa.sync_status() == fa.FA_OK
+        what = f"{'paired' if mode == '1' else 'one-SM'} dK/dV {B,H,N} causal={causal}"
+        for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+            check_grad(f64(g), ref[name], name, what)
+        grads[mode] = (dq.clone(), dk.clone(), dv.clone())
+    monkeypatch.delenv("FA_BWD_PAIR")
+    # dQ comes from the same kernel either way
+    assert torch.equal(grads["0"][0], grads["1"][0])
