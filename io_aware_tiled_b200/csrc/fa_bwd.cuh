@@ -116,11 +116,17 @@ __global__ void __launch_bounds__(DkdvCfg<D>::THREADS, 1)
 
   // Block order: head-major without a mask (the blocks resident together
   // share one head's Q and dO in L2); with the causal mask, the longest key
-  // tiles (the first ones) of every head come first, so the last wave is short.
+  // tiles (the first ones) of every head of a group (causal_head_group) come
+  // first, so the last wave is short.
   const int NKT = (N + C::BK - 1) / C::BK;
   const int BHg = gridDim.x / NKT;
-  const int bh = CAUSAL ? blockIdx.x % BHg : blockIdx.x / NKT;
-  const int kt = CAUSAL ? blockIdx.x / BHg : blockIdx.x - bh * NKT;
+  int bh, kt;
+  if (CAUSAL) {
+    causal_grouped_unit(blockIdx.x, BHg, NKT, causal_head_group(BHg, N, D), bh, kt);
+  } else {
+    bh = blockIdx.x / NKT;
+    kt = blockIdx.x - bh * NKT;
+  }
   const int NQT = (N + C::BQ - 1) / C::BQ;
   const int i0 = CAUSAL ? (kt * C::BK) / C::BQ : 0;  // first query tile that sees these keys
   const int nt = NQT - i0;                           // >= 1: the tile holding query kt*BK exists
@@ -360,11 +366,18 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // Block order as in the dK/dV kernel: head-major without a mask, longest
-  // query tiles (the last ones) of every head first with it.
+  // query tiles (the last ones) of every head of a group first with it.
   const int NQT = (N + C::BQ - 1) / C::BQ;
   const int BHg = gridDim.x / NQT;
-  const int bh = CAUSAL ? blockIdx.x % BHg : blockIdx.x / NQT;
-  const int qt = CAUSAL ? NQT - 1 - blockIdx.x / BHg : blockIdx.x - bh * NQT;
+  int bh, qt;
+  if (CAUSAL) {
+    int r;
+    causal_grouped_unit(blockIdx.x, BHg, NQT, causal_head_group(BHg, N, D), bh, r);
+    qt = NQT - 1 - r;
+  } else {
+    bh = blockIdx.x / NQT;
+    qt = blockIdx.x - bh * NQT;
+  }
   const int NKT = (N + C::BK - 1) / C::BK;
   const int nt = CAUSAL ? min(NKT, (qt * C::BQ + C::BQ - 1) / C::BK + 1) : NKT;
 

@@ -90,8 +90,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Dkdv2Cfg::THREADS, 1
   const int pair = blockIdx.x >> 1;
   const int NKP = (N + 2 * C::BK - 1) / (2 * C::BK);
   const int BHg = (gridDim.x >> 1) / NKP;
-  const int bh = CAUSAL ? pair % BHg : pair / NKP;
-  const int kp = CAUSAL ? pair / BHg : pair - bh * NKP;
+  int bh, kp;
+  if (CAUSAL) {
+    causal_grouped_unit(pair, BHg, NKP, causal_head_group(BHg, N, D), bh, kp);
+  } else {
+    bh = pair / NKP;
+    kp = pair - bh * NKP;
+  }
   const int key0 = kp * 2 * C::BK + static_cast<int>(rank) * C::BK;  // this CTA's first key
   const int NQT = (N + C::BQ - 1) / C::BQ;
   const int i0 = CAUSAL ? (kp * 2 * C::BK) / C::BQ : 0;  // first query tile that sees the pair's keys

@@ -592,6 +592,33 @@ __device__ __forceinline__ float exp2_poly3(float t) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Maximum of the NC (a multiple of 8, >= 32) values of s: 8 independent
+// chains of three-input maxima, then a three-input tree.
+template <int NC>
+__device__ __forceinline__ float row_max(const float (&s)[NC]) {
+  static_assert(NC % 8 == 0 && NC >= 32, "row_max expects a multiple of 8 columns, at least 32");
+  float pm[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) pm[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+  int c = 24;
+#pragma unroll
+  for (; c + 16 <= NC; c += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pm[e] = fmax3(pm[e], s[c + e], s[c + 8 + e]);
+  if (c < NC) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
+  }
+  return fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
   return *reinterpret_cast<uint32_t*>(&v);
@@ -603,6 +630,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // per-worker sums far better than plain round robin.
 __device__ __forceinline__ int serpentine_unit(int k, int w, int W) {
   return k * W + ((k & 1) ? (W - 1 - w) : w);
+}
+
+// Causal block orders of the backward launch the longest blocks first so the
+// last wave is short; across all heads at once, that keeps every head's K and
+// V (or Q and dO) in flight.  Heads therefore go in groups whose K and V
+// (bf16) fit in 64 MiB of the 126 MB L2 (all heads when they fit), longest
+// blocks first inside each group.  Returns the group size.
+__device__ __forceinline__ int causal_head_group(int BH, int N, int D) {
+  const long long per_head = 4ll * N * D;
+  const long long g = (64ll << 20) / per_head;
+  return g >= BH ? BH : (g < 1 ? 1 : static_cast<int>(g));
+}
+// Unit u of that order for units of NR ranks per head (rank 0 = longest):
+// head bh and rank r.
+__device__ __forceinline__ void causal_grouped_unit(int u, int BH, int NR, int G, int& bh, int& r) {
+  const int per_group = G * NR;
+  const int g = u / per_group;
+  const int v = u - g * per_group;
+  const int gh = min(G, BH - g * G);  // heads in this group (the last may be short)
+  r = v / gh;
+  bh = g * G + (v - r * gh);
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -66,8 +66,9 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   // warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 idle; warpgroups 1 and 2: softmax of Q tile 0 and 1
   static constexpr int THREADS = 384;
-  // register split (launch: 384 threads x 168): control warpgroup 56, softmax warpgroups 216 each
-  static constexpr uint32_t REGS_CONTROL = 56, REGS_SOFTMAX = 216;
+  // register split (launch: 384 threads x 168 = 64512): control warpgroup 64,
+  // softmax warpgroups 208 each (128 x 64 + 256 x 208 = 61440)
+  static constexpr uint32_t REGS_CONTROL = 64, REGS_SOFTMAX = 208;
   // one exponential pair in EXP_EMUL_EVERY goes to exp2_poly3 (FMA pipe)
   // instead of the MUFU: 1/4 of them at d = 64, 1/8 at d = 128 (measured best)
   static constexpr int EXP_EMUL_EVERY = (D == 64) ? 4 : 8;
@@ -81,7 +82,8 @@ enum FwdWaitSite : unsigned int {
 // Unit order.  Non-causal: head-major, so the CTAs running at the same time
 // share a few heads' K and V in L2.  Causal: longest units (last query pairs)
 // first across all heads, dealt in serpentine order (serpentine_unit), so the
-// persistent CTAs finish together.
+// persistent CTAs finish together.  (Grouping heads to keep K and V in L2, as
+// the backward does, breaks the global longest-first sort and costs more.)
 __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool causal, int& bh, int& qp) {
   if (causal) {
     const int r = u / BH;
@@ -326,19 +328,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
             if (key >= N || (CAUSAL && key > row)) s[c] = -INFINITY;
           }
         }
-        // row max: 8 independent partial maxima, then a tree (short dependency chains)
-        float pm[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pm[e] = s[e];
-#pragma unroll
-        for (int c = 8; c < NC; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
-#pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
-        const float mx = pm[0];
+        const float mx = row_max<NC>(s);  // 8 independent chains of 3-input maxima
         const float m_new = fmaxf(m_ref, mx * scale_log2);
         const bool need = m_new > m_ref + rescale_log2;
         const bool warp_rescale = __any_sync(0xffffffffu, need);

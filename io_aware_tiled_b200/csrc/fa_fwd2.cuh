@@ -73,7 +73,7 @@ enum Fwd2WaitSite : unsigned int {
 
 // Pair unit u covers query tiles 2*qp (rank 0) and 2*qp+1 (rank 1) of head bh.
 // Non-causal: head-major (concurrent pairs share a few heads' K/V in L2).
-// Causal: longest units first across heads.
+// Causal: longest units first across all heads.
 __device__ __forceinline__ void fwd2_decode_unit(int u, int BH, int NQP, bool causal, int& bh, int& qp) {
   if (causal) {
     const int r = u / BH;
@@ -308,25 +308,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
             if (key >= N || (CAUSAL && key > row)) s[c] = -INFINITY;
           }
         }
-        float pm[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pm[e] = s[e];
-#pragma unroll
-        for (int c = 8; c < 64; c += 8)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pm[e] = fmaxf(pm[e], s[c + e]);
-#pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
+        const float pmax = row_max<64>(s);
         // Row max across the two halves.  The exchange slot alternates with the
         // step, so a slot is rewritten only after the partner has passed the
         // next barrier, i.e. after it read this step's value.  Both halves
         // then hold the same max, hence the same m and rescale decisions.
         float* slot = xmax + (j & 1) * 256;
-        slot[h * 128 + r] = pm[0];
+        slot[h * 128 + r] = pmax;
         named_bar_sync(1, 256);
-        const float mx = fmaxf(pm[0], slot[(1 - h) * 128 + r]);
+        const float mx = fmaxf(pmax, slot[(1 - h) * 128 + r]);
         // Both halves have loaded their S before that barrier, so from here on
         // P may be written over S's columns.
         const float m_new = fmaxf(m_ref, mx * scale_log2);
