@@ -260,7 +260,8 @@ NCU_TRAFFIC_PER_HEAD = {
     "fa_bwd_dkdv_kernel": (270.878720e6 + 103.970816e6) / 64,
     "fa_bwd_dq_kernel": (270.584576e6 + 51.742208e6) / 64,
 }
-NCU_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_device.cuh", "fa_fwd.cuh", "fa_fwd2.cuh")
+NCU_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_bwd2.cuh", "fa_device.cuh", "fa_fwd.cuh", "fa_fwd2.cuh",
+               "fa_unfused.cuh")
 NCU_SOURCES_SHA = "c6d45be6f17046b72e39a06805a2283f364c0f75bcb892c75b6f5959c9e26608"
 
 
