@@ -252,35 +252,37 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # captured with `python bench.py --ncu-case fwd|bwd` (B=4, H=16, N=4096,
 # d=128, non-causal: 64 heads) and divided by the 64 heads; the summaries sit
 # in profiles/.  Each kernel reads its inputs once per head, so the traffic of
-# the bench's 32-head launch is the per-head figure x 32.  SOURCES_SHA is the
-# sha256 of the kernel sources at capture time: once they change the figures
-# no longer describe the kernels and traffic is reported as null.
-NCU_TRAFFIC_PER_HEAD = {
-    "fa_fwd_2sm_kernel": (201.413376e6 + 49.094656e6) / 64,
-    "fa_bwd_dkdv_kernel": (270.878720e6 + 103.970816e6) / 64,
-    "fa_bwd_dq_kernel": (270.584576e6 + 51.742208e6) / 64,
+# the bench's 32-head launch is the per-head figure x 32.  Each entry keeps the
+# sha256 of the sources the kernel is compiled from at capture time: once they
+# change, the figure no longer describes the kernel and traffic is null.
+NCU_TRAFFIC = {
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (201.415168e6 + 51.269120e6) / 64,
+                          "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
+                          "sha256": "94c61c24f4f62b4c19a61f4d9c82f9dda1b8a2b78f43214dd4ac47f54b83e257"},
+    "fa_bwd_dkdv_kernel": {"bytes_per_head": (270.758144e6 + 103.693824e6) / 64,
+                           "sources": ("fa_bwd.cuh", "fa_device.cuh"),
+                           "sha256": "105e14ddf5f946b5e6b5ba46e955de295b09f20301f310c4494f0d2e4e6f0234"},
+    "fa_bwd_dq_kernel": {"bytes_per_head": (270.868736e6 + 52.507392e6) / 64,
+                         "sources": ("fa_bwd.cuh", "fa_device.cuh"),
+                         "sha256": "105e14ddf5f946b5e6b5ba46e955de295b09f20301f310c4494f0d2e4e6f0234"},
 }
-NCU_SOURCES = ("fa_api.cu", "fa_bwd.cuh", "fa_bwd2.cuh", "fa_device.cuh", "fa_fwd.cuh", "fa_fwd2.cuh",
-               "fa_unfused.cuh")
-NCU_SOURCES_SHA = "c6d45be6f17046b72e39a06805a2283f364c0f75bcb892c75b6f5959c9e26608"
 
 
-def kernel_sources_sha() -> str:
+def kernel_sources_sha(sources) -> str:
     import hashlib
     h = hashlib.sha256()
     root = os.path.join(os.path.dirname(os.path.abspath(__file__)), "io_aware_tiled_b200", "csrc")
-    for name in NCU_SOURCES:
+    for name in sources:
         with open(os.path.join(root, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
 def ncu_traffic_per_launch(heads: int) -> dict:
-    """DRAM bytes per launch for `heads` (B*H) heads, by kernel name; empty
-    when the kernel sources changed since the capture."""
-    if kernel_sources_sha() != NCU_SOURCES_SHA:
-        return {}
-    return {n: b * heads for n, b in NCU_TRAFFIC_PER_HEAD.items()}
+    """DRAM bytes per launch for `heads` (B*H) heads, by kernel name, for the
+    kernels whose sources are unchanged since the capture."""
+    return {n: e["bytes_per_head"] * heads for n, e in NCU_TRAFFIC.items()
+            if kernel_sources_sha(e["sources"]) == e["sha256"]}
 
 
 # ---------------------------------------------------------------------------
