@@ -193,6 +193,39 @@ def cpu_baseline(target_s=12.0):
             "host_cpu_count": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
 
 
+def run_oracle_configs():
+    """The oracle (fp64, host cores) timed on every named workload, forward and
+    backward as the workload names them: the whole workload for the small ones,
+    two heads extrapolated to all heads for the long-sequence one (heads are
+    independent), and the single-head workload also on one core.  A reported
+    baseline, not a target.  One JSON line per (workload, mask)."""
+    import oracle
+    from io_aware_tiled_b200.configs import WORKLOADS
+    from io_aware_tiled_b200.inputs import attention_inputs
+    cores = oracle.num_threads()
+    for w in WORKLOADS.values():
+        heads = w.B * w.H
+        timed_heads = 2 if w.N >= 16384 else heads
+        q, k, v, do = attention_inputs(1, timed_heads, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk)
+        args = [t.double().numpy() for t in (q, k, v, do)]
+        for causal in w.causal_modes:
+            for threads in ((cores, 1) if heads == 1 else (cores,)):
+                oracle.set_num_threads(threads)
+                t0 = time.perf_counter()
+                if w.backward:
+                    oracle.backward(*args, causal, w.scale)
+                else:
+                    oracle.forward(*args[:3], causal, w.scale)
+                dt = (time.perf_counter() - t0) * heads / timed_heads
+                flops = w.fwd_flops(causal) + (w.bwd_flops(causal) if w.backward else 0.0)
+                print(json.dumps({"oracle": w.name, "causal": causal, "pass": "fwd+bwd" if w.backward else "fwd",
+                                  "seconds": dt, "tflops": flops / dt / 1e12, "cores": threads,
+                                  "timed_heads": timed_heads, "heads": heads,
+                                  "extrapolated": timed_heads != heads}), flush=True)
+        oracle.set_num_threads(cores)
+    return 0
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -668,16 +701,22 @@ def run_tile_sweep(steps: int, warmup: int):
     return 0
 
 
-def run_ncu_case(case: str, batch: int):
+def run_ncu_case(case: str, batch: int, workload: str | None = None):
     """A few launches of one kernel family, untimed, for ncu captures: the
     headline shape with B=`batch` (B=4: Q, K, V, O, dO are 67 MB each, so the
-    working set exceeds the 126 MB L2).  One warm-up launch, then two."""
+    working set exceeds the 126 MB L2), or a named workload's shape and value
+    spread.  One warm-up launch, then two."""
     import torch
 
     from io_aware_tiled_b200 import fa
+    from io_aware_tiled_b200.configs import WORKLOADS
     from io_aware_tiled_b200.inputs import attention_inputs
     dev = torch.device("cuda", 0)
-    q, k, v, do = (t.to(dev) for t in attention_inputs(batch, 16, 4096, 128, seed=0))
+    if workload:
+        w = WORKLOADS[workload]
+        q, k, v, do = (t.to(dev) for t in attention_inputs(w.B, w.H, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk))
+    else:
+        q, k, v, do = (t.to(dev) for t in attention_inputs(batch, 16, 4096, 128, seed=0))
     causal = case.endswith("causal")
     o, lse = fa.forward(q, k, v, causal)
     ws_unf = torch.empty(fa.unfused_workspace_bytes(*q.shape), dtype=torch.uint8, device=dev) \
@@ -690,7 +729,7 @@ def run_ncu_case(case: str, batch: int):
         else:
             fa.backward(q, k, v, o, do, lse, causal)
     rc = fa.sync_status(dev)
-    print(f"ncu case {case} B={batch}: {fa.status_string(rc)}", flush=True)
+    print(f"ncu case {case} {workload or f'B={batch}'}: {fa.status_string(rc)}", flush=True)
     return 0 if rc == fa.FA_OK else 1
 
 
@@ -704,6 +743,10 @@ def main(argv=None):
     ap.add_argument("--ncu-case", choices=["fwd", "fwd_causal", "bwd", "bwd_causal", "fwd_unfused"], default=None,
                     help="run a few untimed launches for an ncu capture and exit")
     ap.add_argument("--ncu-batch", type=int, default=4)
+    ap.add_argument("--ncu-workload", default=None,
+                    help="run the --ncu-case on this named workload (its B, H, N, d, spread) instead")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="time the fp64 oracle on every named workload on the host cores and exit")
     ap.add_argument("--tile-sweep", action="store_true",
                     help="time the forward for every tile shape the kernels build and exit")
     ap.add_argument("--all-configs", action="store_true",
@@ -713,8 +756,10 @@ def main(argv=None):
         return run_all_configs(max(args.steps, 50), max(args.warmup, 10))
     if args.tile_sweep:
         return run_tile_sweep(max(args.steps, 5), max(args.warmup, 3))
+    if args.oracle_configs:
+        return run_oracle_configs()
     if args.ncu_case:
-        return run_ncu_case(args.ncu_case, args.ncu_batch)
+        return run_ncu_case(args.ncu_case, args.ncu_batch, args.ncu_workload)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
