@@ -354,6 +354,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
 
     fwd_name = fa.forward_kernel_name(d, False)
+    dkdv_name = fa.dkdv_kernel_name(d)
 
     def timed(fn, steps, per_kernel=False):
         """Run fn `steps` times, L2 flushed before each; returns total ms and
@@ -381,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
         if per_kernel:
             kern = {fwd_name: [e[0].elapsed_time(e[1]) for e in kev],
                     "fa_bwd_preprocess_kernel": [e[1].elapsed_time(e[2]) for e in kev],
-                    "fa_bwd_dkdv_kernel": [e[2].elapsed_time(e[3]) for e in kev],
+                    dkdv_name: [e[2].elapsed_time(e[3]) for e in kev],
                     "fa_bwd_dq_kernel": [e[3].elapsed_time(e[4]) for e in kev]}
         return total, kern
 
@@ -455,7 +456,7 @@ def run_ours(args, rank, world, local_rank):
     kavg = {n: sum(v) / len(v) for n, v in kern.items()}
     per_kernel_flops = {  # dense MMA work each kernel performs
         fwd_name: 4.0 * B * H * N * N * d,
-        "fa_bwd_dkdv_kernel": 8.0 * B * H * N * N * d,   # S^T, dP^T, dV, dK
+        dkdv_name: 8.0 * B * H * N * N * d,              # S^T, dP^T, dV, dK
         "fa_bwd_dq_kernel": 6.0 * B * H * N * N * d,     # S, dP, dQ
     }
     traffic = ncu_traffic_per_launch(B * H)

@@ -181,6 +181,17 @@ const char* fa_status_string(int status);
 const char* fa_fwd_kernel_name(int d, int causal);
 
 /*
+ * Name of the dK/dV kernel fa_bwd launches for head size d:
+ * "fa_bwd_dkdv_kernel" (one CTA per 128-key tile, the default),
+ * "fa_bwd_dkdv_persistent_kernel" (persistent CTAs; environment variable
+ * FA_BWD_PERSIST=1) or "fa_bwd_dkdv_2sm_kernel" (CTA pairs, d = 128 only;
+ * FA_BWD_PAIR=1).  All compute the same dK and dV.  NULL when d is not 64 or
+ * 128.  Static string, owned by the library.  For labelling timings and
+ * profiles; the paper has no counterpart.
+ */
+const char* fa_bwd_dkdv_kernel_name(int d);
+
+/*
  * Fault-detection self test.  Launches one tiny kernel that waits on a
  * barrier nothing ever signals, with a wall-clock limit of `limit_us`
  * microseconds (1 .. 10,000,000).  The wait runs out, the kernel records

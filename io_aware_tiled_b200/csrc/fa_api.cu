@@ -9,6 +9,7 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_bwd2.cuh"
+#include "fa_bwd3.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd2.cuh"
 #include "fa_unfused.cuh"
@@ -107,6 +108,10 @@ int device_ready(int* sms, int* pair_clusters = nullptr) {
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, true>, fa::DqCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<false>, fa::Fwd2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<true>, fa::Fwd2Cfg::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<64, false>, fa::Dkdv3Cfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<64, true>, fa::Dkdv3Cfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<128, false>, fa::Dkdv3Cfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<128, true>, fa::Dkdv3Cfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dkdv_2sm_kernel<false>, fa::Dkdv2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_bwd_dkdv_2sm_kernel<true>, fa::Dkdv2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_scores_kernel<64>, fa::UnfScoresCfg<64>::SMEM_BYTES);
@@ -384,6 +389,24 @@ int fa_fwd_unfused(const void* Q, const void* K, const void* V, void* O, float* 
   return launch_status();
 }
 
+// Which dK/dV kernel fa_bwd launches: 1 one CTA per 128-key tile (the
+// default), 0 persistent CTAs (FA_BWD_PERSIST=1; correct, but no faster: 2-6%
+// slower without the mask at N = 4096), 2 CTA pairs (FA_BWD_PAIR=1, d = 128
+// only; correct, but slower: with two S^T/dP^T buffers, tensor memory being
+// full, each tile waits on two cross-SM signals).
+static int bwd_dkdv_form(int d) {
+  const char* pair_env = getenv("FA_BWD_PAIR");
+  if (d == 128 && pair_env && strcmp(pair_env, "1") == 0) return 2;
+  const char* persist_env = getenv("FA_BWD_PERSIST");
+  return (persist_env && strcmp(persist_env, "1") == 0) ? 0 : 1;
+}
+
+const char* fa_bwd_dkdv_kernel_name(int d) {
+  if (d != 64 && d != 128) return nullptr;
+  static const char* names[3] = {"fa_bwd_dkdv_persistent_kernel", "fa_bwd_dkdv_kernel", "fa_bwd_dkdv_2sm_kernel"};
+  return names[bwd_dkdv_form(d)];
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (check_sizes(B, H, N, d)) return 0;
   const size_t dbytes = static_cast<size_t>(B) * H * N * 4;
@@ -450,28 +473,28 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   };
   const int grid_kv = BH * ((N + 127) / 128);
   const int grid_q = BH * ((N + 127) / 128);
-  // FA_BWD_PAIR=1 runs dK/dV on CTA pairs (256 keys per pair, d = 128) for
-  // comparisons: correct, but slower than one SM per 128 keys, because with
-  // two S^T/dP^T buffers (tensor memory is full) each tile waits on two
-  // cross-SM signals.
-  const char* bwd_pair_env = getenv("FA_BWD_PAIR");
-  const bool bwd_pair = d == 128 && bwd_pair_env && strcmp(bwd_pair_env, "1") == 0;
+  const int dkdv_form = bwd_dkdv_form(d);
+  const bool bwd_pair = dkdv_form == 2;
   CUtensorMap mq32, mdo32;
   if (bwd_pair && (!make_map(&mq32, Q, BH, N, d, 32) || !make_map(&mdo32, dO, BH, N, d, 32)))
     return encode_failed();
   const int grid_kv2 = 2 * BH * ((N + 255) / 256);
+  const bool persist = dkdv_form == 0;
+  const int grid_kvp = grid_kv < sms ? grid_kv : sms;
   if (d == 64) {
     const long long threads = rows * 8;
     mark(0);
     fa::fa_bwd_preprocess_kernel<64><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(o, dob, Dvec, rows);
     mark(1);
     if (causal) {
-      fa::fa_bwd_dkdv_kernel<64, true><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      (persist ? fa::fa_bwd_dkdv_persistent_kernel<64, true><<<grid_kvp, fa::Dkdv3Cfg<64>::THREADS, fa::Dkdv3Cfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
+                 : fa::fa_bwd_dkdv_kernel<64, true><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
       mark(2);
       fa::fa_bwd_dq_kernel<64, true><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
       mark(3);
     } else {
-      fa::fa_bwd_dkdv_kernel<64, false><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      (persist ? fa::fa_bwd_dkdv_persistent_kernel<64, false><<<grid_kvp, fa::Dkdv3Cfg<64>::THREADS, fa::Dkdv3Cfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
+                 : fa::fa_bwd_dkdv_kernel<64, false><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
       mark(2);
       fa::fa_bwd_dq_kernel<64, false><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
       mark(3);
@@ -485,7 +508,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
       if (bwd_pair)
         fa::fa_bwd_dkdv_2sm_kernel<true><<<grid_kv2, fa::Dkdv2Cfg::THREADS, fa::Dkdv2Cfg::SMEM_BYTES, s>>>(mq32, mdo32, mq64, mdo64, mk128, mv128, LSE, Dvec, dk, dv, N, sc, sl2);
       else
-        fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+        (persist ? fa::fa_bwd_dkdv_persistent_kernel<128, true><<<grid_kvp, fa::Dkdv3Cfg<128>::THREADS, fa::Dkdv3Cfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
+                 : fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
       mark(2);
       fa::fa_bwd_dq_kernel<128, true><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
       mark(3);
@@ -493,7 +517,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
       if (bwd_pair)
         fa::fa_bwd_dkdv_2sm_kernel<false><<<grid_kv2, fa::Dkdv2Cfg::THREADS, fa::Dkdv2Cfg::SMEM_BYTES, s>>>(mq32, mdo32, mq64, mdo64, mk128, mv128, LSE, Dvec, dk, dv, N, sc, sl2);
       else
-        fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+        (persist ? fa::fa_bwd_dkdv_persistent_kernel<128, false><<<grid_kvp, fa::Dkdv3Cfg<128>::THREADS, fa::Dkdv3Cfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
+                 : fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
       mark(2);
       fa::fa_bwd_dq_kernel<128, false><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
       mark(3);

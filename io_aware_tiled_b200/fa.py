@@ -75,6 +75,8 @@ def load_library(build_if_missing: bool = True):
         lib.fa_fwd_unfused_workspace_bytes.restype = sz
         lib.fa_fwd_unfused.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
         lib.fa_fwd_unfused.restype = i
+        lib.fa_bwd_dkdv_kernel_name.argtypes = [i]
+        lib.fa_bwd_dkdv_kernel_name.restype = ctypes.c_char_p
         lib.fa_fwd_kernel_name.argtypes = [i, i]
         lib.fa_fwd_kernel_name.restype = ctypes.c_char_p
         lib.fa_bwd_set_phase_events.argtypes = [vp, vp, vp, vp]
@@ -101,6 +103,15 @@ def forward_kernel_name(d: int, causal: bool) -> str:
     name = load_library().fa_fwd_kernel_name(int(d), int(bool(causal)))
     if name is None:
         raise RuntimeError(f"no forward kernel for d={d} on this device")
+    return name.decode()
+
+
+def dkdv_kernel_name(d: int) -> str:
+    """Name of the dK/dV kernel `backward` launches for head size d
+    (fa_bwd_dkdv_kernel_name)."""
+    name = load_library().fa_bwd_dkdv_kernel_name(int(d))
+    if name is None:
+        raise RuntimeError(f"no dK/dV kernel for d={d}")
     return name.decode()
 
 

@@ -25,7 +25,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == {"fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_sync_status", "fa_last_error_word",
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
                           "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name",
-                          "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes"}
+                          "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes", "fa_bwd_dkdv_kernel_name"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:
@@ -132,6 +132,21 @@ def test_unfused_rejects_bad_arguments(lib):
     assert _unf(lib, ws=3 * A) == EWS              # workspace aliases V
     if not torch.cuda.is_available():
         assert _unf(lib) == EDEV
+
+
+def test_dkdv_kernel_name_follows_the_settings(monkeypatch):
+    # pure host logic: no device needed
+    monkeypatch.delenv("FA_BWD_PAIR", raising=False)
+    monkeypatch.delenv("FA_BWD_PERSIST", raising=False)
+    assert fa.dkdv_kernel_name(128) == "fa_bwd_dkdv_kernel"
+    assert fa.dkdv_kernel_name(64) == "fa_bwd_dkdv_kernel"
+    monkeypatch.setenv("FA_BWD_PERSIST", "1")
+    assert fa.dkdv_kernel_name(128) == "fa_bwd_dkdv_persistent_kernel"
+    monkeypatch.setenv("FA_BWD_PAIR", "1")
+    assert fa.dkdv_kernel_name(128) == "fa_bwd_dkdv_2sm_kernel"
+    assert fa.dkdv_kernel_name(64) == "fa_bwd_dkdv_persistent_kernel"
+    with pytest.raises(RuntimeError):
+        fa.dkdv_kernel_name(96)
 
 
 def test_selftest_rejects_bad_limit(lib):
