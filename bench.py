@@ -15,6 +15,11 @@ no collective on the data path); rank 0 prints the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the only other place this
 script runs it) on a bounded sample of the same workload.
+
+Other modes (each prints JSON lines and exits): --all-configs times every
+named workload; --tile-sweep times every forward tile shape the kernels build
+and the rescale thresholds; --oracle-configs times the oracle on every named
+workload; --ncu-case [--ncu-workload] runs a few untimed launches for ncu.
 """
 from __future__ import annotations
 
