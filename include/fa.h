@@ -86,7 +86,12 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  * Workspace: caller-owned device buffer of at least fa_bwd_workspace_bytes()
  *      bytes, 16-byte aligned; its contents on entry do not matter.
  * Launches, in order on `stream`: the D = rowsum(dO * O) pass, the dK/dV
- * kernel, the dQ kernel.  P is recomputed as exp(S - LSE).
+ * kernel, the dQ kernel.  P is recomputed as exp(S - LSE).  The dK/dV kernel
+ * is one CTA per 128-key tile by default; the environment variables
+ * FA_BWD_PERSIST=1 (persistent CTAs) and FA_BWD_PAIR=1 (CTA pairs, d = 128)
+ * select other forms for comparisons (fa_bwd_dkdv_kernel_name); all give the
+ * same dK and dV.  dQ has its own kernel and no atomics: results are
+ * deterministic.
  */
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
            void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
