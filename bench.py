@@ -18,8 +18,8 @@ script runs it) on a bounded sample of the same workload.
 
 Other modes (each prints JSON lines and exits): --all-configs times every
 named workload; --tile-sweep times every forward tile shape the kernels build
-and the rescale thresholds; --oracle-configs times the oracle on every named
-workload; --ncu-case [--ncu-workload] runs a few untimed launches for ncu.
+and the rescale thresholds; --ncu-case [--ncu-workload] runs a few untimed
+launches for ncu.
 """
 from __future__ import annotations
 
@@ -196,39 +196,6 @@ def cpu_baseline(target_s=12.0):
     return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{reps} x one head (B=1,H=1,N=4096,d=128) fwd+bwd non-causal, fp64, {total_t:.1f} s",
             "host_cpu_count": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
-
-
-def run_oracle_configs():
-    """The oracle (fp64, host cores) timed on every named workload, forward and
-    backward as the workload names them: the whole workload for the small ones,
-    two heads extrapolated to all heads for the long-sequence one (heads are
-    independent), and the single-head workload also on one core.  A reported
-    baseline, not a target.  One JSON line per (workload, mask)."""
-    import oracle
-    from io_aware_tiled_b200.configs import WORKLOADS
-    from io_aware_tiled_b200.inputs import attention_inputs
-    cores = oracle.num_threads()
-    for w in WORKLOADS.values():
-        heads = w.B * w.H
-        timed_heads = 2 if w.N >= 16384 else heads
-        q, k, v, do = attention_inputs(1, timed_heads, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk)
-        args = [t.double().numpy() for t in (q, k, v, do)]
-        for causal in w.causal_modes:
-            for threads in ((cores, 1) if heads == 1 else (cores,)):
-                oracle.set_num_threads(threads)
-                t0 = time.perf_counter()
-                if w.backward:
-                    oracle.backward(*args, causal, w.scale)
-                else:
-                    oracle.forward(*args[:3], causal, w.scale)
-                dt = (time.perf_counter() - t0) * heads / timed_heads
-                flops = w.fwd_flops(causal) + (w.bwd_flops(causal) if w.backward else 0.0)
-                print(json.dumps({"oracle": w.name, "causal": causal, "pass": "fwd+bwd" if w.backward else "fwd",
-                                  "seconds": dt, "tflops": flops / dt / 1e12, "cores": threads,
-                                  "timed_heads": timed_heads, "heads": heads,
-                                  "extrapolated": timed_heads != heads}), flush=True)
-        oracle.set_num_threads(cores)
-    return 0
 
 
 def run_reference(args, rank, world):
@@ -751,8 +718,6 @@ def main(argv=None):
     ap.add_argument("--ncu-batch", type=int, default=4)
     ap.add_argument("--ncu-workload", default=None,
                     help="run the --ncu-case on this named workload (its B, H, N, d, spread) instead")
-    ap.add_argument("--oracle-configs", action="store_true",
-                    help="time the fp64 oracle on every named workload on the host cores and exit")
     ap.add_argument("--tile-sweep", action="store_true",
                     help="time the forward for every tile shape the kernels build and exit")
     ap.add_argument("--all-configs", action="store_true",
@@ -762,8 +727,6 @@ def main(argv=None):
         return run_all_configs(max(args.steps, 50), max(args.warmup, 10))
     if args.tile_sweep:
         return run_tile_sweep(max(args.steps, 5), max(args.warmup, 3))
-    if args.oracle_configs:
-        return run_oracle_configs()
     if args.ncu_case:
         return run_ncu_case(args.ncu_case, args.ncu_batch, args.ncu_workload)
 
