@@ -317,8 +317,8 @@ def run_ours(args, rank, world, local_rank):
     def fwd(causal):
         fa.forward(qd, kd, vd, causal, out=o, lse=lse)
 
-    def bwd(causal):
-        fa.backward(qd, kd, vd, o, dod, lse, causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+    def bwd(causal, deterministic=False):
+        fa.backward(qd, kd, vd, o, dod, lse, causal, workspace=ws, dq=dq, dk=dk, dv=dv, deterministic=deterministic)
 
     def barrier():
         if world > 1:
@@ -326,7 +326,9 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
 
     fwd_name = fa.forward_kernel_name(d, False)
-    dkdv_name = fa.dkdv_kernel_name(d)
+    pre_name, main_bwd_name, last_bwd_name = fa.backward_kernel_names(d)
+
+    step_times = []  # per-step ms of each timed() call, in call order
 
     def timed(fn, steps, per_kernel=False):
         """Run fn `steps` times, L2 flushed before each; returns total ms and
@@ -349,13 +351,15 @@ def run_ours(args, rank, world, local_rank):
                 fn()
             ev[i][1].record(stream)
         barrier()
-        total = sum(a.elapsed_time(b) for a, b in ev)
+        per_step = [a.elapsed_time(b) for a, b in ev]
+        total = sum(per_step)
+        step_times.append(per_step)
         kern = None
         if per_kernel:
             kern = {fwd_name: [e[0].elapsed_time(e[1]) for e in kev],
-                    "fa_bwd_preprocess_kernel": [e[1].elapsed_time(e[2]) for e in kev],
-                    dkdv_name: [e[2].elapsed_time(e[3]) for e in kev],
-                    "fa_bwd_dq_kernel": [e[3].elapsed_time(e[4]) for e in kev]}
+                    pre_name: [e[1].elapsed_time(e[2]) for e in kev],
+                    main_bwd_name: [e[2].elapsed_time(e[3]) for e in kev],
+                    last_bwd_name: [e[3].elapsed_time(e[4]) for e in kev]}
         return total, kern
 
     # warm-up (also the status check: a kernel timeout would show here)
@@ -371,9 +375,16 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(dev)
     with clocks:
         main_ms, kern = timed(None, args.steps, per_kernel=True)
+        main_steps = step_times[-1]
         fwd_ms, _ = timed(lambda: fwd(False), args.steps)
+        fwd_steps = step_times[-1]
         fwdc_ms, _ = timed(lambda: fwd(True), args.steps)
+        fwdc_steps = step_times[-1]
         stepc_ms, _ = timed(lambda: (fwd(True), bwd(True)), args.steps)
+        stepc_steps = step_times[-1]
+        # the deterministic backward form (a separate dQ kernel), for comparison
+        stepd_ms, _ = timed(lambda: (fwd(False), bwd(False, True)), args.steps)
+        stepd_steps = step_times[-1]
     # the standard (unfused) forward of the same batch, for the HBM-traffic
     # comparison: S and P through HBM (outside the clock sampling window)
     ws_unf = torch.empty(fa.unfused_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
@@ -387,6 +398,7 @@ def run_ours(args, rank, world, local_rank):
     fwd_ms = max_over_ranks(fwd_ms, world, dev)
     fwdc_ms = max_over_ranks(fwdc_ms, world, dev)
     stepc_ms = max_over_ranks(stepc_ms, world, dev)
+    stepd_ms = max_over_ranks(stepd_ms, world, dev)
     rc = fa.sync_status(dev)
     if rc != fa.FA_OK:
         raise RuntimeError(f"library status {fa.status_string(rc)}")
@@ -421,6 +433,12 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
     d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
 
+    # every other named workload (forward, forward + backward), median and best
+    wclocks = ClockSampler(dev)
+    with wclocks:
+        wlines = time_workloads(args.workload_steps, max(args.warmup, 3), dev,
+                                reduce_max=lambda x: max_over_ranks(x, world, dev), skip=(WORKLOAD,))
+
     peaks = _peaks()
     step_flops = f_nc + b_nc
     value = whole_job_tflops(world, step_flops, args.steps, main_ms)
@@ -428,8 +446,14 @@ def run_ours(args, rank, world, local_rank):
     kavg = {n: sum(v) / len(v) for n, v in kern.items()}
     per_kernel_flops = {  # dense MMA work each kernel performs
         fwd_name: 4.0 * B * H * N * N * d,
-        dkdv_name: 8.0 * B * H * N * N * d,              # S^T, dP^T, dV, dK
-        "fa_bwd_dq_kernel": 6.0 * B * H * N * N * d,     # S, dP, dQ
+        main_bwd_name: 10.0 * B * H * N * N * d,         # S^T, dP^T, dV, dK, dQ^T
+    }
+    # bytes the memory-bound passes must move: the D pass reads O and dO,
+    # writes D and zeroes the fp32 dQ accumulator; the convert pass reads the
+    # accumulator and writes bf16 dQ
+    per_kernel_bytes = {
+        pre_name: 2.0 * B * H * N * d * 2 + 4.0 * B * H * N + 4.0 * B * H * N * d,
+        last_bwd_name: 4.0 * B * H * N * d + 2.0 * B * H * N * d,
     }
     traffic = ncu_traffic_per_launch(B * H)
     dom = max(kavg, key=kavg.get)
@@ -439,16 +463,16 @@ def run_ours(args, rank, world, local_rank):
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": traffic.get(dom), "peak_kind": f"bf16 burst, {peaks['source']}"}
     else:
-        bytes_pre = 2.0 * B * H * N * d * 2 + 4.0 * B * H * N
-        ach = bytes_pre / (kavg[dom] * 1e-3) / 1e9
+        ach = per_kernel_bytes[dom] / (kavg[dom] * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / peaks["hbm_gbs"], "traffic": traffic.get(dom), "peak_kind": f"hbm copy, {peaks['source']}"}
     kernels = {n: {"ms": kavg[n],
                    "tflops": (per_kernel_flops[n] / (kavg[n] * 1e-3) / 1e12) if n in per_kernel_flops else None,
                    "traffic": traffic.get(n)}
                for n in kavg}
-    kernels["fa_bwd_preprocess_kernel"]["gbs"] = (2.0 * B * H * N * d * 2 + 4.0 * B * H * N) / (
-        kavg["fa_bwd_preprocess_kernel"] * 1e-3) / 1e9
+    for n, nb in per_kernel_bytes.items():
+        kernels[n]["gbs"] = nb / (kavg[n] * 1e-3) / 1e9
+        kernels[n]["frac_of_hbm"] = kernels[n]["gbs"] / peaks["hbm_gbs"]
 
     out = None
     if rank == 0:
@@ -460,13 +484,27 @@ def run_ours(args, rank, world, local_rank):
                        "inputs": "i.i.d. N(0,1) bf16 from seed 0 (+rank)", "l2": "256 MiB written between timed steps",
                        "parallelism": f"independent batch per GPU x{world}"},
             "frac_of_peak": value / peak,
+            "median_ms_per_step": statistics.median(main_steps), "best_ms_per_step": min(main_steps),
+            "value_median": world * step_flops / (statistics.median(main_steps) * 1e-3) / 1e12,
+            "value_best": world * step_flops / (min(main_steps) * 1e-3) / 1e12,
             "legs": {
-                "fwd_noncausal": {"tflops": world * f_nc * args.steps / (fwd_ms * 1e-3) / 1e12,
-                                  "ms": fwd_ms / args.steps},
-                "fwd_causal": {"tflops": world * f_c * args.steps / (fwdc_ms * 1e-3) / 1e12,
-                               "ms": fwdc_ms / args.steps},
-                "fwd_bwd_causal": {"tflops": world * (f_c + b_c) * args.steps / (stepc_ms * 1e-3) / 1e12,
-                                   "ms": stepc_ms / args.steps},
+                "fwd_noncausal": _leg(world * f_nc, fwd_ms, args.steps, fwd_steps, peak),
+                "fwd_causal": _leg(world * f_c, fwdc_ms, args.steps, fwdc_steps, peak),
+                "fwd_bwd_causal": _leg(world * (f_c + b_c), stepc_ms, args.steps, stepc_steps, peak),
+                # backward alone: the step minus the forward of the same mask
+                "bwd_noncausal": {"tflops": world * b_nc / ((main_ms - fwd_ms) / args.steps * 1e-3) / 1e12,
+                                  "ms": (main_ms - fwd_ms) / args.steps,
+                                  "frac_of_measured_peak": world * b_nc / ((main_ms - fwd_ms) / args.steps * 1e-3)
+                                  / 1e12 / peak, "how": "mean fwd+bwd step minus mean forward"},
+                "fwd_bwd_noncausal_deterministic": _leg(world * (f_nc + b_nc), stepd_ms, args.steps, stepd_steps,
+                                                        peak),
+                "bwd_noncausal_deterministic": {
+                    "tflops": world * b_nc / ((stepd_ms - fwd_ms) / args.steps * 1e-3) / 1e12,
+                    "ms": (stepd_ms - fwd_ms) / args.steps, "how": "mean fwd+bwd step minus mean forward"},
+                "bwd_causal": {"tflops": world * b_c / ((stepc_ms - fwdc_ms) / args.steps * 1e-3) / 1e12,
+                               "ms": (stepc_ms - fwdc_ms) / args.steps,
+                               "frac_of_measured_peak": world * b_c / ((stepc_ms - fwdc_ms) / args.steps * 1e-3)
+                               / 1e12 / peak, "how": "mean fwd+bwd step minus mean forward"},
                 # standard attention: S (fp16) and P (bf16) written and read
                 # once each through HBM; bytes per head as in the pages'
                 # table: Q, K, V, S, P read; S, P, O written
@@ -485,6 +523,8 @@ def run_ours(args, rank, world, local_rank):
                     "api": "io_aware_tiled_b200.host_pipeline.forward_backward_host",
                     "serial_value": world * step_flops * e2e_steps / (e2e_serial_ms * 1e-3) / 1e12,
                     "serial_ms_per_step": e2e_serial_ms / e2e_steps},
+            "workloads": wlines,
+            "workloads_clocks": wclocks.summary(),
             "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
             "peaks": peaks,
@@ -492,20 +532,32 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
-def run_all_configs(steps: int, warmup: int):
+def _leg(flops_per_step, total_ms, steps, per_step_ms, peak):
+    """TFLOP/s of one timed leg: mean over the steps, plus median and best."""
+    med, best = statistics.median(per_step_ms), min(per_step_ms)
+    mean = total_ms / steps
+    return {"tflops": flops_per_step / (mean * 1e-3) / 1e12, "ms": mean,
+            "tflops_median": flops_per_step / (med * 1e-3) / 1e12, "median_ms": med,
+            "tflops_best": flops_per_step / (best * 1e-3) / 1e12, "best_ms": best,
+            "frac_of_measured_peak": flops_per_step / (mean * 1e-3) / 1e12 / peak}
+
+
+def time_workloads(steps: int, warmup: int, dev, reduce_max=lambda x: x, skip=()):
     """Every named workload on one GPU: forward (each mask it names) and, where
     it names one, forward + backward; CUDA events around each call, the L2
     flushed before each (the small single-head workload also without the
-    flush), median and best of `steps` calls after `warmup`.  One JSON line
-    per (workload, mask, pass)."""
+    flush, and replayed from a CUDA graph), median and best of `steps` calls
+    after `warmup`.  Returns one dict per (workload, mask, pass, timing form).
+    `reduce_max` maps a local time to the max over ranks (identity on one GPU);
+    every rank makes the same calls in the same order."""
     import torch
 
     from io_aware_tiled_b200 import fa
     from io_aware_tiled_b200.configs import WORKLOADS
     from io_aware_tiled_b200.inputs import attention_inputs
-    dev = torch.device("cuda", 0)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     peak = _peaks()["bf16_tflops"]
+    lines = []
 
     def time_calls(fn, do_flush):
         for _ in range(warmup):
@@ -523,15 +575,18 @@ def run_all_configs(steps: int, warmup: int):
         rc = fa.sync_status(dev)
         if rc != fa.FA_OK:
             raise RuntimeError(f"library status {fa.status_string(rc)}")
-        return statistics.median(ts), min(ts)
+        return reduce_max(statistics.median(ts)), reduce_max(min(ts))
 
     for w in WORKLOADS.values():
+        if w.name in skip:
+            continue
         q, k, v, do = (t.to(dev) for t in attention_inputs(w.B, w.H, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk))
         o = torch.empty_like(q)
         lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
         dq, dk, dv = (torch.empty_like(q) for _ in range(3))
         ws = torch.empty(fa.workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
         io_bytes = w.B * w.H * w.N * (4 * w.d * 2 + 4)  # Q, K, V read; O written; LSE written
+        small = w.B * w.H * w.N <= 4096
         for causal in w.causal_modes:
             passes = [("fwd", lambda: fa.forward(q, k, v, causal, out=o, lse=lse), w.fwd_flops(causal))]
             if w.backward:
@@ -540,9 +595,10 @@ def run_all_configs(steps: int, warmup: int):
                                                                dq=dq, dk=dk, dv=dv)),
                                w.fwd_flops(causal) + w.bwd_flops(causal)))
             for name, fn, flops in passes:
-                for do_flush in ((True, False) if w.N * w.B * w.H <= 4096 else (True,)):
+                forms = [("eager", True)] + ([("eager", False)] if small else [])
+                for launch, do_flush in forms:
                     med, best = time_calls(fn, do_flush)
-                    line = {"workload": w.name, "causal": causal, "pass": name,
+                    line = {"workload": w.name, "causal": causal, "pass": name, "launch": launch,
                             "kernel": fa.forward_kernel_name(w.d, causal),
                             "median_us": med * 1e3, "best_us": best * 1e3,
                             "tflops_median": flops / (med * 1e-3) / 1e12, "tflops_best": flops / (best * 1e-3) / 1e12,
@@ -551,8 +607,9 @@ def run_all_configs(steps: int, warmup: int):
                             "steps": steps, "warmup": warmup}
                     if name == "fwd":
                         line["gbs_median"] = io_bytes / (med * 1e-3) / 1e9
-                    print(json.dumps(line), flush=True)
-                if w.B * w.H * w.N <= 4096:
+                        line["gbs_best"] = io_bytes / (best * 1e-3) / 1e9
+                    lines.append(line)
+                if small:
                     # latency-bound: the same call replayed from a CUDA graph
                     # (no host-side work between the events)
                     fn()
@@ -562,15 +619,27 @@ def run_all_configs(steps: int, warmup: int):
                         fn()
                     for do_flush in (True, False):
                         med, best = time_calls(graph.replay, do_flush)
-                        print(json.dumps({"workload": w.name, "causal": causal, "pass": name, "launch": "graph replay",
-                                          "median_us": med * 1e3, "best_us": best * 1e3,
-                                          "tflops_median": flops / (med * 1e-3) / 1e12,
-                                          "gbs_median": io_bytes / (med * 1e-3) / 1e9 if name == "fwd" else None,
-                                          "l2": "flushed before each call" if do_flush else "warm (no flush)",
-                                          "steps": steps, "warmup": warmup}), flush=True)
+                        lines.append({"workload": w.name, "causal": causal, "pass": name, "launch": "graph replay",
+                                      "median_us": med * 1e3, "best_us": best * 1e3,
+                                      "tflops_median": flops / (med * 1e-3) / 1e12,
+                                      "tflops_best": flops / (best * 1e-3) / 1e12,
+                                      "gbs_median": io_bytes / (med * 1e-3) / 1e9 if name == "fwd" else None,
+                                      "gbs_best": io_bytes / (best * 1e-3) / 1e9 if name == "fwd" else None,
+                                      "l2": "flushed before each call" if do_flush else "warm (no flush)",
+                                      "steps": steps, "warmup": warmup})
                     del graph
         del q, k, v, do, o, lse, dq, dk, dv, ws
         torch.cuda.empty_cache()
+    del flush
+    torch.cuda.empty_cache()
+    return lines
+
+
+def run_all_configs(steps: int, warmup: int):
+    """time_workloads on cuda:0, one JSON line per entry."""
+    import torch
+    for line in time_workloads(steps, warmup, torch.device("cuda", 0)):
+        print(json.dumps(line), flush=True)
     return 0
 
 
@@ -706,6 +775,27 @@ def run_ncu_case(case: str, batch: int, workload: str | None = None):
     return 0 if rc == fa.FA_OK else 1
 
 
+def launch_ranks(n: int, impl: str, argv: list) -> int:
+    """`--gpus N` without a launcher: start N ranks of this script with
+    torch.distributed.run on this node (rendezvous on 127.0.0.1, one rank per
+    GPU), wait for them and return their exit status.  The GPU arm needs N
+    visible CUDA devices; the reference arm runs on the host cores (rank 0
+    only) and needs none."""
+    import socket
+    if impl == "ours":
+        import torch
+        have = torch.cuda.device_count()
+        if have < n:
+            print(f"bench.py: --gpus {n} needs {n} visible CUDA devices, found {have}", file=sys.stderr)
+            return 2
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -713,6 +803,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload-steps", type=int, default=20,
+                    help="timed calls per leg of the other named workloads in the default run")
     ap.add_argument("--ncu-case", choices=["fwd", "fwd_causal", "bwd", "bwd_causal", "fwd_unfused"], default=None,
                     help="run a few untimed launches for an ncu capture and exit")
     ap.add_argument("--ncu-batch", type=int, default=4)
@@ -730,9 +822,15 @@ def main(argv=None):
     if args.ncu_case:
         return run_ncu_case(args.ncu_case, args.ncu_batch, args.ncu_workload)
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(args.gpus, args.impl, sys.argv[1:] if argv is None else list(argv))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU "
+              f"(torchrun --nproc-per-node {args.gpus}) or pass --gpus {world}", file=sys.stderr)
+        return 2
 
     if args.impl == "reference":
         return run_reference(args, rank, world)

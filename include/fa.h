@@ -72,9 +72,10 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
            int causal, float scale, void* stream);
 
 /*
- * Bytes of device workspace fa_bwd needs for these sizes (the fp32 row
- * vector D = rowsum(dO * O), [B,H,N], rounded up to 256 bytes).  Returns 0
- * for invalid sizes.
+ * Bytes of device workspace fa_bwd needs for these sizes: the fp32 row vector
+ * D = rowsum(dO * O) ([B,H,N], rounded up to 256 bytes) followed by the fp32
+ * dQ accumulator ([B,H,N,d]).  Enough for fa_bwd_deterministic too, which
+ * uses only the D part.  Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -84,18 +85,35 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *      from fa_fwd with the same causal flag and scale.
  * Out: dQ, dK, dV [B,H,N,d] bf16.
  * Workspace: caller-owned device buffer of at least fa_bwd_workspace_bytes()
- *      bytes, 16-byte aligned; its contents on entry do not matter.
- * Launches, in order on `stream`: the D = rowsum(dO * O) pass, the dK/dV
- * kernel, the dQ kernel.  P is recomputed as exp(S - LSE).  The dK/dV kernel
- * is one CTA per 128-key tile by default; the environment variables
- * FA_BWD_PERSIST=1 (persistent CTAs) and FA_BWD_PAIR=1 (CTA pairs, d = 128)
- * select other forms for comparisons (fa_bwd_dkdv_kernel_name); all give the
- * same dK and dV.  dQ has its own kernel and no atomics: results are
- * deterministic.
+ *      bytes, 16-byte aligned, not overlapping any other argument; its
+ *      contents on entry do not matter.
+ * Three launches, in order on `stream`: the D = rowsum(dO * O) pass (which
+ * also zeroes the dQ accumulator); fa_bwd_fused_kernel, one CTA per 128 keys
+ * of a head, which recomputes P = exp(S - LSE) tile by tile and forms all
+ * five products of the gradient -- S, dP, dV, dK and the tile's share of dQ,
+ * added into the fp32 accumulator by the bulk-copy engine; and a pass that
+ * writes dQ = bf16(scale * accumulator).  dK and dV are accumulated in a
+ * fixed order and are deterministic; the partial sums of dQ arrive in an
+ * order that varies from run to run, so dQ can differ in its last bits
+ * between runs (fa_bwd_deterministic does not).
  */
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
            void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd with bit-reproducible results: the same arguments and outputs, but
+ * dQ gets its own kernel (one CTA per 128 query rows) that recomputes S and
+ * dP instead of adding partial sums, so every output is written once by one
+ * CTA and repeated calls give identical bits.  It performs seven tensor-core
+ * products per tile pair instead of five and is slower.  Launches: the D
+ * pass, fa_bwd_dkdv_kernel, fa_bwd_dq_kernel.  The workspace must hold at
+ * least the D part (4 * B*H*N bytes rounded up to 256); a buffer of
+ * fa_bwd_workspace_bytes() always suffices.
+ */
+int fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                         const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal,
+                         float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fa_bwd for callers that cannot allocate device memory -- for example a
@@ -103,15 +121,19 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
  * code running under a memory pool that must not grow.  The paper has no
  * counterpart to this entry point.
  *
- * Same arguments, semantics and outputs as fa_bwd, minus the workspace: the
+ * Same arguments, semantics and outputs as fa_bwd_deterministic (the form
+ * whose only scratch is the D vector), minus the workspace: the
  * D = rowsum(dO * O) vector lives in a fixed array inside the library
  * (FA_NOALLOC_MAX_ROWS fp32 entries = 4 MiB, held on every GPU that loads the
  * library until the process exits).  The call itself allocates nothing.
+ * Results are bit-identical to fa_bwd_deterministic's.
  *  - Sizes: B*H*N must not exceed FA_NOALLOC_MAX_ROWS, else FA_ERR_TOO_LARGE
  *    (nothing is launched).
  *  - Set-up: the first call on each device looks up the array's device address
  *    (with that device current); make that first call before any stream
- *    capture.
+ *    capture.  The address is remembered per device together with the CUDA
+ *    context it belongs to; after a device reset (a new primary context) the
+ *    next call looks it up again.
  *  - The array is shared by every call on a device and keeps the last call's
  *    contents; each call overwrites the part it uses before reading it.  Calls
  *    that overlap on the GPU (different streams, no ordering between them) race
@@ -143,11 +165,14 @@ unsigned int fa_last_error_word(void);
 int fa_last_cuda_error(void);
 
 /*
- * Optional per-kernel timing of fa_bwd (profiling aid).  When set, fa_bwd
- * records the four cudaEvent_t handles (passed as void*) on its stream:
- * e0 before the D pass, e1 before the dK/dV kernel, e2 before the dQ
- * kernel, e3 after it.  Events belong to the caller and must stay valid while
- * set; pass four NULLs to stop.  The setting is process-wide.
+ * Optional per-kernel timing of the backward (profiling aid).  When set,
+ * fa_bwd, fa_bwd_deterministic and fa_bwd_noalloc record the four
+ * cudaEvent_t handles (passed as void*) on their stream: e0 before the D
+ * pass, e1 before the second launch (fa_bwd_fused_kernel, or
+ * fa_bwd_dkdv_kernel for the deterministic form), e2 before the third (the
+ * dQ conversion, or fa_bwd_dq_kernel), e3 after it.  Events belong to the
+ * caller and must stay valid while set; pass four NULLs to stop.  The setting
+ * is process-wide.
  */
 void fa_bwd_set_phase_events(void* e0, void* e1, void* e2, void* e3);
 
@@ -186,13 +211,11 @@ const char* fa_status_string(int status);
 const char* fa_fwd_kernel_name(int d, int causal);
 
 /*
- * Name of the dK/dV kernel fa_bwd launches for head size d:
- * "fa_bwd_dkdv_kernel" (one CTA per 128-key tile, the default),
- * "fa_bwd_dkdv_persistent_kernel" (persistent CTAs; environment variable
- * FA_BWD_PERSIST=1) or "fa_bwd_dkdv_2sm_kernel" (CTA pairs, d = 128 only;
- * FA_BWD_PAIR=1).  All compute the same dK and dV.  NULL when d is not 64 or
- * 128.  Static string, owned by the library.  For labelling timings and
- * profiles; the paper has no counterpart.
+ * Name of the kernel that computes dK and dV in fa_bwd for head size d:
+ * "fa_bwd_fused_kernel" (which also forms the dQ partial sums).
+ * fa_bwd_deterministic runs "fa_bwd_dkdv_kernel" instead.  NULL when d is
+ * not 64 or 128.  Static string, owned by the library.  For labelling
+ * timings and profiles; the paper has no counterpart.
  */
 const char* fa_bwd_dkdv_kernel_name(int d);
 

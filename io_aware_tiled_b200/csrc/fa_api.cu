@@ -8,8 +8,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
-#include "fa_bwd2.cuh"
-#include "fa_bwd3.cuh"
+#include "fa_bwd_fused.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd2.cuh"
 #include "fa_unfused.cuh"
@@ -37,7 +36,7 @@ EncodeTiledFn encode_fn() {
 // rows x 1 head, 128-byte swizzle.  Rows past N read as zero within the head.
 int g_last_encode_error = 0;  // CUresult of the last failed tensor-map encode (diagnosis)
 
-bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+bool encode_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     g_last_encode_error = -1;
@@ -52,6 +51,42 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_ro
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) g_last_encode_error = static_cast<int>(r);
   return r == CUDA_SUCCESS;
+}
+
+// Encoded tensor maps, remembered by (address, heads, rows, head size, box
+// rows): a map holds only the address and the layout, so a later call on the
+// same tensor -- or on a new tensor of the same shape at the same address --
+// reuses it instead of encoding it again.  A small table, replaced round-robin.
+struct MapEntry {
+  const void* base = nullptr;
+  int BH = 0, N = 0, d = 0, box_rows = 0;
+  CUtensorMap map;
+};
+constexpr int kMapCache = 64;
+MapEntry g_maps[kMapCache];
+int g_maps_next = 0;
+std::mutex g_maps_mu;
+
+bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int box_rows) {
+  {
+    std::lock_guard<std::mutex> lock(g_maps_mu);
+    for (const MapEntry& e : g_maps)
+      if (e.base == base && e.BH == BH && e.N == N && e.d == d && e.box_rows == box_rows) {
+        *m = e.map;
+        return true;
+      }
+  }
+  if (!encode_map(m, base, BH, N, d, box_rows)) return false;
+  std::lock_guard<std::mutex> lock(g_maps_mu);
+  MapEntry& e = g_maps[g_maps_next];
+  g_maps_next = (g_maps_next + 1) % kMapCache;
+  e.base = base;
+  e.BH = BH;
+  e.N = N;
+  e.d = d;
+  e.box_rows = box_rows;
+  e.map = *m;
+  return true;
 }
 
 constexpr int kMaxDevices = 64;
@@ -108,12 +143,10 @@ int device_ready(int* sms, int* pair_clusters = nullptr) {
     ok = ok && set_smem(fa::fa_bwd_dq_kernel<128, true>, fa::DqCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<false>, fa::Fwd2Cfg::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_fwd_2sm_kernel<true>, fa::Fwd2Cfg::SMEM_BYTES);
-    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<64, false>, fa::Dkdv3Cfg<64>::SMEM_BYTES);
-    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<64, true>, fa::Dkdv3Cfg<64>::SMEM_BYTES);
-    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<128, false>, fa::Dkdv3Cfg<128>::SMEM_BYTES);
-    ok = ok && set_smem(fa::fa_bwd_dkdv_persistent_kernel<128, true>, fa::Dkdv3Cfg<128>::SMEM_BYTES);
-    ok = ok && set_smem(fa::fa_bwd_dkdv_2sm_kernel<false>, fa::Dkdv2Cfg::SMEM_BYTES);
-    ok = ok && set_smem(fa::fa_bwd_dkdv_2sm_kernel<true>, fa::Dkdv2Cfg::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_fused_kernel<64, false>, fa::FusedCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_fused_kernel<64, true>, fa::FusedCfg<64>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_fused_kernel<128, false>, fa::FusedCfg<128>::SMEM_BYTES);
+    ok = ok && set_smem(fa::fa_bwd_fused_kernel<128, true>, fa::FusedCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_scores_kernel<64>, fa::UnfScoresCfg<64>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_scores_kernel<128>, fa::UnfScoresCfg<128>::SMEM_BYTES);
     ok = ok && set_smem(fa::fa_unf_pv_kernel<64>, fa::UnfPvCfg<64>::SMEM_BYTES);
@@ -171,15 +204,64 @@ int encode_failed() {
 }
 std::mutex g_events_mu;
 
-bool is_device_ptr(const void* p) {
+// Device-memory allocations already seen, as address ranges per device: a
+// pointer inside one of them is device memory of that device without asking
+// the driver again (the check costs a driver call per pointer otherwise).
+// Ranges come from cuMemGetAddressRange on pointers the runtime reported as
+// device memory of the current device.  Freeing an allocation does not
+// remove its range; the addresses of freed device memory are only handed out
+// again for device memory.
+struct RangeEntry {
+  uintptr_t lo = 0, hi = 0;
+  int dev = -1;
+};
+constexpr int kRangeCache = 256;
+RangeEntry g_ranges[kRangeCache];
+int g_ranges_next = 0;
+std::mutex g_ranges_mu;
+
+using GetAddressRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+GetAddressRangeFn address_range_fn() {
+  static GetAddressRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetAddressRangeFn>(p);
+  });
+  return fn;
+}
+
+// True if [p, p + bytes) is device (or managed) memory of the current device.
+bool is_device_ptr(const void* p, size_t bytes = 1) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p), hi = lo + (bytes ? bytes : 1);
+  {
+    std::lock_guard<std::mutex> lock(g_ranges_mu);
+    for (const RangeEntry& e : g_ranges)
+      if (e.dev == dev && lo >= e.lo && hi <= e.hi) return true;
+  }
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
-  int dev = 0;
-  cudaGetDevice(&dev);
-  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+  if (!((a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev)) return false;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  GetAddressRangeFn fn = address_range_fn();
+  if (fn && fn(&base, &size, static_cast<CUdeviceptr>(lo)) == CUDA_SUCCESS && size > 0) {
+    std::lock_guard<std::mutex> lock(g_ranges_mu);
+    RangeEntry& e = g_ranges[g_ranges_next];
+    g_ranges_next = (g_ranges_next + 1) % kRangeCache;
+    e.lo = static_cast<uintptr_t>(base);
+    e.hi = static_cast<uintptr_t>(base) + size;
+    e.dev = dev;
+  }
+  return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -275,7 +357,8 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
     return FA_ERR_INVALID_ARG;
   int sms = 0, pair_clusters[2] = {0, 0};
   if ((rc = device_ready(&sms, pair_clusters))) return rc;
-  if (!is_device_ptr(Q) || !is_device_ptr(K) || !is_device_ptr(V) || !is_device_ptr(O) || !is_device_ptr(LSE))
+  if (!is_device_ptr(Q, tbytes) || !is_device_ptr(K, tbytes) || !is_device_ptr(V, tbytes) ||
+      !is_device_ptr(O, tbytes) || !is_device_ptr(LSE, lbytes))
     return FA_ERR_UNSUPPORTED_DEVICE;
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
@@ -362,8 +445,8 @@ int fa_fwd_unfused(const void* Q, const void* K, const void* V, void* O, float* 
     return FA_ERR_WORKSPACE;
   int sms = 0;
   if ((rc = device_ready(&sms))) return rc;
-  if (!is_device_ptr(Q) || !is_device_ptr(K) || !is_device_ptr(V) || !is_device_ptr(O) || !is_device_ptr(LSE) ||
-      !is_device_ptr(workspace))
+  if (!is_device_ptr(Q, tbytes) || !is_device_ptr(K, tbytes) || !is_device_ptr(V, tbytes) ||
+      !is_device_ptr(O, tbytes) || !is_device_ptr(LSE, lbytes) || !is_device_ptr(workspace, need))
     return FA_ERR_UNSUPPORTED_DEVICE;
   const int Nr = static_cast<int>(nt * 128);
   CUtensorMap mq, mk, mp, mv;
@@ -389,41 +472,38 @@ int fa_fwd_unfused(const void* Q, const void* K, const void* V, void* O, float* 
   return launch_status();
 }
 
-// Which dK/dV kernel fa_bwd launches: 1 one CTA per 128-key tile (the
-// default), 0 persistent CTAs (FA_BWD_PERSIST=1; correct, but no faster: 2-6%
-// slower without the mask at N = 4096), 2 CTA pairs (FA_BWD_PAIR=1, d = 128
-// only; correct, but slower: with two S^T/dP^T buffers, tensor memory being
-// full, each tile waits on two cross-SM signals).
-static int bwd_dkdv_form(int d) {
-  const char* pair_env = getenv("FA_BWD_PAIR");
-  if (d == 128 && pair_env && strcmp(pair_env, "1") == 0) return 2;
-  const char* persist_env = getenv("FA_BWD_PERSIST");
-  return (persist_env && strcmp(persist_env, "1") == 0) ? 0 : 1;
-}
-
 const char* fa_bwd_dkdv_kernel_name(int d) {
   if (d != 64 && d != 128) return nullptr;
-  static const char* names[3] = {"fa_bwd_dkdv_persistent_kernel", "fa_bwd_dkdv_kernel", "fa_bwd_dkdv_2sm_kernel"};
-  return names[bwd_dkdv_form(d)];
+  return "fa_bwd_fused_kernel";
 }
 
-size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (check_sizes(B, H, N, d)) return 0;
+// Workspace of the backward: D (fp32 [B*H*N], padded to 256 bytes), then the
+// fp32 dQ accumulator [B*H*N*d] of the fused form.
+static size_t bwd_d_bytes(int B, int H, int N) {
   const size_t dbytes = static_cast<size_t>(B) * H * N * 4;
   return (dbytes + 255) & ~static_cast<size_t>(255);
 }
 
-int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
-           void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, void* workspace,
-           size_t workspace_bytes, void* stream) {
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d)) return 0;
+  return bwd_d_bytes(B, H, N) + static_cast<size_t>(B) * H * N * d * 4;
+}
+
+// The backward in either form.  fused: one kernel computes dK, dV and the dQ
+// partials (fp32 accumulator in the workspace), then a convert pass; else the
+// deterministic form: dK/dV kernel and a dQ kernel that recomputes S and dP.
+// `need` is the workspace the form uses (validated against workspace_bytes).
+static int bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                      void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
+                      void* workspace, size_t workspace_bytes, void* stream, bool fused) {
   int rc = check_sizes(B, H, N, d);
   if (rc) return rc;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
       !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
     return FA_ERR_ALIGNMENT;
-  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_bytes(B, H, N, d))
-    return FA_ERR_WORKSPACE;
+  const size_t need = fused ? fa_bwd_workspace_bytes(B, H, N, d) : bwd_d_bytes(B, H, N);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
   bool scale_ok = false;
   const float sc = effective_scale(scale, d, &scale_ok);
   if (!scale_ok) return FA_ERR_INVALID_ARG;
@@ -434,7 +514,7 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   const Range outs[4] = {{(uintptr_t)dQ, (uintptr_t)dQ + tbytes},
                          {(uintptr_t)dK, (uintptr_t)dK + tbytes},
                          {(uintptr_t)dV, (uintptr_t)dV + tbytes},
-                         {(uintptr_t)workspace, (uintptr_t)workspace + fa_bwd_workspace_bytes(B, H, N, d)}};
+                         {(uintptr_t)workspace, (uintptr_t)workspace + need}};
   for (int a = 0; a < 4; ++a) {
     for (int b = 0; b < 6; ++b)
       if (overlaps(outs[a], ins[b])) return a == 3 ? FA_ERR_WORKSPACE : FA_ERR_INVALID_ARG;
@@ -444,18 +524,21 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   int sms = 0;
   if ((rc = device_ready(&sms))) return rc;
   const void* ptrs[10] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
-  for (const void* p : ptrs)
-    if (!is_device_ptr(p)) return FA_ERR_UNSUPPORTED_DEVICE;
+  const size_t sizes[10] = {tbytes, tbytes, tbytes, tbytes, tbytes, lbytes, tbytes, tbytes, tbytes, need};
+  for (int i = 0; i < 10; ++i)
+    if (!is_device_ptr(ptrs[i], sizes[i])) return FA_ERR_UNSUPPORTED_DEVICE;
   const int BH = B * H;
   CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128, mk64, mv64;
   if (!make_map(&mq64, Q, BH, N, d, 64) || !make_map(&mdo64, dO, BH, N, d, 64) ||
-      !make_map(&mk128, K, BH, N, d, 128) || !make_map(&mv128, V, BH, N, d, 128) ||
-      !make_map(&mq128, Q, BH, N, d, 128) || !make_map(&mdo128, dO, BH, N, d, 128) ||
-      !make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64))
+      !make_map(&mk128, K, BH, N, d, 128) || !make_map(&mv128, V, BH, N, d, 128))
+    return encode_failed();
+  if (!fused && (!make_map(&mq128, Q, BH, N, d, 128) || !make_map(&mdo128, dO, BH, N, d, 128) ||
+                 !make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64)))
     return encode_failed();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   clear_stale_error();
   float* Dvec = static_cast<float*>(workspace);
+  float* dqacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + bwd_d_bytes(B, H, N));
   const long long rows = static_cast<long long>(BH) * N;
   const float sl2 = sc * fa::kLog2e;
   auto* dq = static_cast<__nv_bfloat16*>(dQ);
@@ -473,58 +556,60 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   };
   const int grid_kv = BH * ((N + 127) / 128);
   const int grid_q = BH * ((N + 127) / 128);
-  const int dkdv_form = bwd_dkdv_form(d);
-  const bool bwd_pair = dkdv_form == 2;
-  CUtensorMap mq32, mdo32;
-  if (bwd_pair && (!make_map(&mq32, Q, BH, N, d, 32) || !make_map(&mdo32, dO, BH, N, d, 32)))
-    return encode_failed();
-  const int grid_kv2 = 2 * BH * ((N + 255) / 256);
-  const bool persist = dkdv_form == 0;
-  const int grid_kvp = grid_kv < sms ? grid_kv : sms;
+  const unsigned grid_pre = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
+  const unsigned grid_cvt = static_cast<unsigned>((rows * d / 8 + 255) / 256);
+  mark(0);
   if (d == 64) {
-    const long long threads = rows * 8;
-    mark(0);
-    fa::fa_bwd_preprocess_kernel<64><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(o, dob, Dvec, rows);
-    mark(1);
-    if (causal) {
-      (persist ? fa::fa_bwd_dkdv_persistent_kernel<64, true><<<grid_kvp, fa::Dkdv3Cfg<64>::THREADS, fa::Dkdv3Cfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
-                 : fa::fa_bwd_dkdv_kernel<64, true><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
+    if (fused) {
+      fa::fa_bwd_preprocess_kernel<64, true><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows, dqacc);
+      mark(1);
+      if (causal) fa::fa_bwd_fused_kernel<64, true><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      else fa::fa_bwd_fused_kernel<64, false><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
       mark(2);
-      fa::fa_bwd_dq_kernel<64, true><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
-      mark(3);
+      fa::fa_bwd_dq_convert_kernel<<<grid_cvt, 256, 0, s>>>(dqacc, dq, rows * d / 8, sc);
     } else {
-      (persist ? fa::fa_bwd_dkdv_persistent_kernel<64, false><<<grid_kvp, fa::Dkdv3Cfg<64>::THREADS, fa::Dkdv3Cfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
-                 : fa::fa_bwd_dkdv_kernel<64, false><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
+      fa::fa_bwd_preprocess_kernel<64><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows);
+      mark(1);
+      if (causal) fa::fa_bwd_dkdv_kernel<64, true><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      else fa::fa_bwd_dkdv_kernel<64, false><<<grid_kv, fa::DkdvCfg<64>::THREADS, fa::DkdvCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
       mark(2);
-      fa::fa_bwd_dq_kernel<64, false><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
-      mark(3);
+      if (causal) fa::fa_bwd_dq_kernel<64, true><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
+      else fa::fa_bwd_dq_kernel<64, false><<<grid_q, fa::DqCfg<64>::THREADS, fa::DqCfg<64>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
     }
   } else {
-    const long long threads = rows * 16;
-    mark(0);
-    fa::fa_bwd_preprocess_kernel<128><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(o, dob, Dvec, rows);
-    mark(1);
-    if (causal) {
-      if (bwd_pair)
-        fa::fa_bwd_dkdv_2sm_kernel<true><<<grid_kv2, fa::Dkdv2Cfg::THREADS, fa::Dkdv2Cfg::SMEM_BYTES, s>>>(mq32, mdo32, mq64, mdo64, mk128, mv128, LSE, Dvec, dk, dv, N, sc, sl2);
-      else
-        (persist ? fa::fa_bwd_dkdv_persistent_kernel<128, true><<<grid_kvp, fa::Dkdv3Cfg<128>::THREADS, fa::Dkdv3Cfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
-                 : fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
+    if (fused) {
+      fa::fa_bwd_preprocess_kernel<128, true><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows, dqacc);
+      mark(1);
+      if (causal) fa::fa_bwd_fused_kernel<128, true><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      else fa::fa_bwd_fused_kernel<128, false><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
       mark(2);
-      fa::fa_bwd_dq_kernel<128, true><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
-      mark(3);
+      fa::fa_bwd_dq_convert_kernel<<<grid_cvt, 256, 0, s>>>(dqacc, dq, rows * d / 8, sc);
     } else {
-      if (bwd_pair)
-        fa::fa_bwd_dkdv_2sm_kernel<false><<<grid_kv2, fa::Dkdv2Cfg::THREADS, fa::Dkdv2Cfg::SMEM_BYTES, s>>>(mq32, mdo32, mq64, mdo64, mk128, mv128, LSE, Dvec, dk, dv, N, sc, sl2);
-      else
-        (persist ? fa::fa_bwd_dkdv_persistent_kernel<128, false><<<grid_kvp, fa::Dkdv3Cfg<128>::THREADS, fa::Dkdv3Cfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, BH, N, sc, sl2)
-                 : fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2));
+      fa::fa_bwd_preprocess_kernel<128><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows);
+      mark(1);
+      if (causal) fa::fa_bwd_dkdv_kernel<128, true><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
+      else fa::fa_bwd_dkdv_kernel<128, false><<<grid_kv, fa::DkdvCfg<128>::THREADS, fa::DkdvCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, N, sc, sl2);
       mark(2);
-      fa::fa_bwd_dq_kernel<128, false><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
-      mark(3);
+      if (causal) fa::fa_bwd_dq_kernel<128, true><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
+      else fa::fa_bwd_dq_kernel<128, false><<<grid_q, fa::DqCfg<128>::THREADS, fa::DqCfg<128>::SMEM_BYTES, s>>>(mq128, mk64, mv64, mdo128, LSE, Dvec, dq, N, sc, sl2);
     }
   }
+  mark(3);
   return launch_status();
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, workspace, workspace_bytes, stream,
+                    true);
+}
+
+int fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                         const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal,
+                         float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, workspace, workspace_bytes, stream,
+                    false);
 }
 
 static unsigned int g_last_error_word = 0;
@@ -538,8 +623,12 @@ void fa_bwd_set_phase_events(void* e0, void* e1, void* e2, void* e3) {
 }
 
 int fa_sync_status(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int>(e);
+    return FA_ERR_LAUNCH;
+  }
   unsigned int word = 0;
   if (cudaMemcpyFromSymbol(&word, fa::g_error_word, sizeof(word)) != cudaSuccess) return FA_ERR_LAUNCH;
   if (word != 0) {
@@ -593,7 +682,26 @@ namespace {
 // kernels get the device address from cudaGetSymbolAddress below.
 __device__ __align__(256) float g_noalloc_d[FA_NOALLOC_MAX_ROWS];
 void* g_noalloc_addr[kMaxDevices] = {};
+void* g_noalloc_ctx[kMaxDevices] = {};  // the CUDA context each address belongs to
 std::mutex g_noalloc_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+// The current thread's CUDA context (the device's primary context once the
+// runtime has bound it), or null.
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
 }  // namespace
 
 extern "C" int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -607,10 +715,19 @@ extern "C" int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const
     cudaGetLastError();
     return FA_ERR_UNSUPPORTED_DEVICE;
   }
+  // Binds the device's primary context to this thread if it has none yet, so
+  // that the context looked up below is the one the kernels will run in.
+  if (cudaSetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_UNSUPPORTED_DEVICE;
+  }
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {  // set-up, once per device, with that device current
+    void* ctx = current_context();
+    // set-up, once per device (and again after a device reset gave it a new
+    // context), with that device current
+    if (!g_noalloc_addr[dev] || ctx != g_noalloc_ctx[dev]) {
       void* p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_d);
       if (e != cudaSuccess || !p) {
@@ -619,11 +736,12 @@ extern "C" int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const
         return FA_ERR_LAUNCH;
       }
       g_noalloc_addr[dev] = p;
+      g_noalloc_ctx[dev] = ctx;
     }
     scratch = g_noalloc_addr[dev];
   }
-  // D is written in full by the first kernel before anything reads it, so the
-  // array needs no clearing between calls.
-  return fa_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, scratch,
-                static_cast<size_t>(FA_NOALLOC_MAX_ROWS) * sizeof(float), stream);
+  // The deterministic form needs only D, which its first kernel writes in full
+  // before anything reads it, so the array needs no clearing between calls.
+  return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, scratch,
+                    static_cast<size_t>(FA_NOALLOC_MAX_ROWS) * sizeof(float), stream, false);
 }

@@ -30,17 +30,25 @@
 namespace fa {
 
 // ---------------------------------------------------------------------------
-// D_i = sum_c dO_ic * O_ic  (fp32), one group of D/8 threads per row
+// D_i = sum_c dO_ic * O_ic  (fp32), one group of D/8 threads per row.  With
+// ZERO the same pass also clears the row of the fp32 dQ accumulator that the
+// fused backward adds into (8 floats per thread).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool ZERO = false>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ O,
                                                                  const __nv_bfloat16* __restrict__ dO,
-                                                                 float* __restrict__ Dout, long long rows) {
+                                                                 float* __restrict__ Dout, long long rows,
+                                                                 float* __restrict__ dQacc = nullptr) {
   constexpr int G = D / 8;  // threads per row; each reads 16 bytes of O and of dO
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long row = gid / G;
   const int part = static_cast<int>(gid % G);
   float acc = 0.f;
+  if (ZERO && row < rows) {
+    float4* z = reinterpret_cast<float4*>(dQacc + row * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (row < rows) {
     const uint4 a = *reinterpret_cast<const uint4*>(O + row * D + part * 8);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);

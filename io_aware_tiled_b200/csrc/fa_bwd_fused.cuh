@@ -1,0 +1,446 @@
+// fa_bwd_fused.cuh -- the backward of tiled, IO-aware exact attention as five
+// tensor-core products per tile (sm_100a).
+//
+// The backward keeps only O and the per-row statistic and recomputes the
+// attention weights tile by tile ("图解Flash Attention运算原理", 总结:
+// Recomputation keeps the softmax statistics and recomputes P when needed):
+// P_ij = exp(S_ij - LSE_i).  The gradients of the loss sum(dO * O) (the
+// analytic gradient of the definition; the pages do not print it):
+//   D_i = sum_c dO_ic O_ic                 (over the bf16 O given)
+//   dV_j = sum_i P_ij dO_i,  dP_ij = dO_i . V_j,  dS_ij = P_ij (dP_ij - D_i)
+//   dK_j = scale sum_i dS_ij Q_i,  dQ_i = scale sum_j dS_ij K_j
+//
+// One CTA per (head, 128-key tile) computes, for every 64-row query tile that
+// can see its keys, all five products: S^T = K Q^T and dP^T = V dO^T into
+// tensor memory, P^T and dS^T from them, dV += P^T dO and dK += dS^T Q with
+// dV, dK accumulating in tensor memory over the whole loop, and the tile's
+// contribution to dQ, dQ_t^T = K^T dS_t^T (d x 64, fp32).  Every key tile of
+// a head adds into the same rows of dQ, so that partial goes to an fp32
+// accumulator in global memory through the bulk-copy engine's reduce-add
+// (element-wise fp32 adds performed in L2, from a shared-memory staging
+// tile).  Three launches in all:
+//   1. fa_bwd_preprocess_kernel<D, true>: D, and zeros into the accumulator;
+//   2. fa_bwd_fused_kernel: dK, dV (bf16, written once) and the dQ partials;
+//   3. fa_bwd_dq_convert_kernel: dQ = bf16(scale * accumulator).
+// The order in which key tiles' partials reach a row of the accumulator is
+// not fixed, so dQ can differ in the last bits from run to run; dK and dV
+// are accumulated in a fixed order.  (fa_bwd.cuh holds the deterministic
+// form: a separate dQ kernel that recomputes S and dP, seven products.)
+//
+// Warp roles (384 threads, three warpgroups):
+//   warp 0       TMA: K and V tiles once; Q and dO tiles through ST stages;
+//                LSE*log2(e) and D of each query tile into shared memory.
+//   warp 1       tcgen05.mma issue (one elected lane), commits.
+//   warps 4-7    softmax gradient: thread = key row.  Reads S^T and dP^T
+//                from tensor memory, writes P^T and dS^T (bf16) back over
+//                S^T's columns (the A operands of dV and dK) and dS^T also to
+//                shared memory (the B operand of dQ^T).
+//   warps 8-11   dQ drain: thread = column c of d.  Reads dQ_t^T from tensor
+//                memory, stores it as a [64 queries][d] fp32 tile in shared
+//                memory and issues the bulk reduce-add of that tile into the
+//                accumulator rows of the query tile.
+// Tensor memory (512 columns): S^T/P^T/dS^T double buffer [0, 128) (64 each:
+// S^T fp32, then P^T in its first 32 and dS^T in its next 32 columns as packed
+// bf16); dP^T double buffer [128, 256), reused for dQ_t^T once the softmax
+// gradient has read dP^T; dV [256, 256+d); dK [256+d, 256+2d).  At d = 64
+// the dQ^T product runs with M = 128 over the adjacent K and V tiles (rows
+// 64..127 of its result, V^T dS^T, are never read), which keeps every MMA in
+// the M = 128 form.
+#pragma once
+
+#include "fa_device.cuh"
+
+namespace fa {
+
+template <int D, int ST_ = ((D == 128) ? 2 : 4), int NDQ_ = 2>
+struct FusedCfg {
+  static constexpr int BK = 128;                      // keys per CTA (MMA M of S^T, dP^T, dV, dK)
+  static constexpr int BQ = 64;                       // queries per tile
+  static constexpr int CH = D / 64;
+  static constexpr int KCHUNK = BK * 128;             // one 64-column chunk of the key tile
+  static constexpr int QCHUNK = BQ * 128;             // one 64-column chunk of a query tile
+  static constexpr int K_TILE = BK * D * 2;
+  static constexpr int Q_TILE = BQ * D * 2;
+  static constexpr int DS_TILE = BK * BQ * 2;         // dS^T: 128 key rows of 64 bf16 (one swizzled chunk)
+  static constexpr int DQ_TILE = BQ * D * 4;          // dQ partial staging: [64 queries][d] fp32
+  static constexpr int ST = ST_;                      // Q / dO stages
+  static constexpr int NDQ = NDQ_;                    // dQ staging buffers
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + K_TILE;        // adjacent to K: the d = 64 dQ^T product reads both
+  static constexpr int OFF_Q = OFF_V + K_TILE;
+  static constexpr int OFF_DO = OFF_Q + ST * Q_TILE;
+  static constexpr int OFF_DS = OFF_DO + ST * Q_TILE;
+  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;
+  static constexpr int OFF_LSE = OFF_DQ + NDQ * DQ_TILE;  // ST x BQ floats (LSE * log2 e)
+  static constexpr int OFF_DD = OFF_LSE + ST * BQ * 4;    // ST x BQ floats (D)
+  static constexpr int OFF_BAR = OFF_DD + ST * BQ * 4;
+  static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = 1 + ST, B_S_FULL = 1 + 2 * ST,
+                       B_P_FULL = B_S_FULL + 2, B_DQ_FULL = B_P_FULL + 2, B_DQ_EMPTY = B_DQ_FULL + 2,
+                       B_STG_FREE = B_DQ_EMPTY + 2, B_STG_FULL = B_STG_FREE + NDQ, B_DKV_FULL = B_STG_FULL + NDQ;
+  static constexpr int NUM_BARS = B_DKV_FULL + 1;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;  // + room to align the base to 1024
+  static_assert(SMEM_BYTES <= 232448, "shared memory of the fused backward exceeds 227 KB");
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 384;
+  // register split (launch: 384 x 168 = 64512): control 64 and dQ drain 160
+  // (both decrease: never above the 168 of the launch), softmax gradient 256
+  // (128 x 480 = 61440)
+  static constexpr uint32_t REGS_CONTROL = 64, REGS_GRAD = 256, REGS_DRAIN = 160;
+  static_assert(REGS_CONTROL <= 168 && REGS_DRAIN <= 168 && 128 * (REGS_CONTROL + REGS_GRAD + REGS_DRAIN) <= 64512,
+                "register split must fit the registers of the launch");
+};
+
+enum FusedWaitSite : unsigned int {
+  BF_PROD_QE = 64, BF_MMA_KV, BF_MMA_Q, BF_MMA_DQE, BF_MMA_P, BF_SM_S, BF_SM_Q, BF_SM_DKV, BF_DR_DQ, BF_DR_FREE,
+  BF_DR_FULL
+};
+
+// Query tile of the it-th step of key tile kt.  With the mask the steps start
+// at the first query tile that sees the keys (i0) and walk up.  Without it
+// every key tile of a head sees all nt query tiles; key tile kt starts at query
+// tile 2kt (mod nt), so the CTAs of a head that run at the same time add their
+// dQ partials into different rows of the accumulator.
+template <bool CAUSAL>
+__device__ __forceinline__ int fused_query_tile(int it, int i0, int nt, int kt) {
+  if (CAUSAL) return i0 + it;
+  int q = it + 2 * kt;
+  q %= nt;
+  return q;
+}
+
+template <int D, bool CAUSAL, int ST_ = ((D == 128) ? 2 : 4), int NDQ_ = 2>
+__global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
+    fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                        const float* __restrict__ LSE, const float* __restrict__ Dvec,
+                        __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+                        float* __restrict__ dQacc, int N, float scale, float scale_log2) {
+  using C = FusedCfg<D, ST_, NDQ_>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sQ = sbase + C::OFF_Q, sdO = sbase + C::OFF_DO;
+  const uint32_t sDS = sbase + C::OFF_DS, sDQ = sbase + C::OFF_DQ;
+  float* sLSE = reinterpret_cast<float*>(smem + C::OFF_LSE);
+  float* sDD = reinterpret_cast<float*>(smem + C::OFF_DD);
+  const uint32_t bars = sbase + C::OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Block order: head-major without the mask; with it, the longest key tiles
+  // (the first ones) of every head of an L2-sized group first.
+  const int NKT = (N + C::BK - 1) / C::BK;
+  const int BHg = gridDim.x / NKT;
+  int bh, kt;
+  if (CAUSAL) {
+    causal_grouped_unit(blockIdx.x, BHg, NKT, causal_head_group(BHg, N, D), bh, kt);
+  } else {
+    bh = blockIdx.x / NKT;
+    kt = blockIdx.x - bh * NKT;
+  }
+  const int NQT = (N + C::BQ - 1) / C::BQ;
+  const int i0 = CAUSAL ? (kt * C::BK) / C::BQ : 0;
+  const int nt = NQT - i0;  // >= 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars + 8 * C::B_KV_FULL, 1);
+    for (int s = 0; s < C::ST; ++s) {
+      mbar_init(bars + 8 * (C::B_Q_FULL + s), 33);  // expect_tx arrive + 32 lanes writing LSE and D
+      mbar_init(bars + 8 * (C::B_Q_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars + 8 * (C::B_S_FULL + b), 1);
+      mbar_init(bars + 8 * (C::B_P_FULL + b), 128);
+      mbar_init(bars + 8 * (C::B_DQ_FULL + b), 1);
+      mbar_init(bars + 8 * (C::B_DQ_EMPTY + b), 128);
+    }
+    for (int b = 0; b < C::NDQ; ++b) {
+      mbar_init(bars + 8 * (C::B_STG_FREE + b), 1);    // the issuing thread: the buffer's last reduce has read it
+      mbar_init(bars + 8 * (C::B_STG_FULL + b), 128);  // every drain thread: its column is stored
+    }
+    mbar_init(bars + 8 * C::B_DKV_FULL, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    regs_dec<C::REGS_CONTROL>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- loads (whole warp)
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmdO);
+        mbar_arrive_expect_tx(bars + 8 * C::B_KV_FULL, 2 * C::K_TILE);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_3d(sK + c * C::KCHUNK, &tmK, bars + 8 * C::B_KV_FULL, c * 64, kt * C::BK, bh);
+          tma_load_3d(sV + c * C::KCHUNK, &tmV, bars + 8 * C::B_KV_FULL, c * 64, kt * C::BK, bh);
+        }
+      }
+      for (int it = 0; it < nt; ++it) {
+        const int st = it % C::ST;
+        const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
+        const bool ok = mbar_wait(bars + 8 * (C::B_Q_EMPTY + st), ((it / C::ST) & 1) ^ 1, BF_PROD_QE);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bars + 8 * (C::B_Q_FULL + st), 2 * C::Q_TILE);
+          for (int c = 0; c < C::CH; ++c) {
+            tma_load_3d(sQ + st * C::Q_TILE + c * C::QCHUNK, &tmQ, bars + 8 * (C::B_Q_FULL + st), c * 64,
+                        qi * C::BQ, bh);
+            tma_load_3d(sdO + st * C::Q_TILE + c * C::QCHUNK, &tmdO, bars + 8 * (C::B_Q_FULL + st), c * 64,
+                        qi * C::BQ, bh);
+          }
+        }
+#pragma unroll
+        for (int e = lane; e < C::BQ; e += 32) {
+          const int q = qi * C::BQ + e;
+          const bool valid = q < N;
+          sLSE[st * C::BQ + e] = valid ? LSE[static_cast<size_t>(bh) * N + q] * kLog2e : INFINITY;
+          sDD[st * C::BQ + e] = valid ? Dvec[static_cast<size_t>(bh) * N + q] : 0.f;
+        }
+        mbar_arrive(bars + 8 * (C::B_Q_FULL + st));
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issue (whole warp, one elected lane)
+      constexpr uint32_t IDESC_T = idesc_bf16(128, C::BQ, false, false);  // S^T, dP^T: M=128 keys, N=64
+      constexpr uint32_t IDESC_G = idesc_bf16(128, D, false, true);        // dV, dK: B MN-major
+      constexpr uint32_t IDESC_DQ = idesc_bf16(128, C::BQ, true, true);    // dQ^T: A and B MN-major
+      auto issue_t = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+        const uint32_t hi = sdesc_hi(1024);
+        const uint64_t a0 = sdesc_make(sdesc_lo(a_smem, 16), hi), b0 = sdesc_make(sdesc_lo(b_smem, 16), hi);
+        if (D == 128)
+          mma_ss_k128(d_tmem, a0, sdesc_make(sdesc_lo(a_smem + C::KCHUNK, 16), hi), b0,
+                      sdesc_make(sdesc_lo(b_smem + C::QCHUNK, 16), hi), IDESC_T, 0u);
+        else
+          mma_ss_k64(d_tmem, a0, b0, IDESC_T, 0u);
+      };
+      auto issue_g = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
+        mma_ts_k64(d_tmem, a_tmem, sdesc_make(sdesc_lo(b_smem, C::QCHUNK), sdesc_hi(1024)), IDESC_G,
+                   acc ? 1u : 0u);
+      };
+      // dQ^T = K^T dS^T: A = the key tile read MN-major (M = d columns, two
+      // 64-column chunks KCHUNK apart; at d = 64 the second chunk is the V
+      // tile), B = dS^T read MN-major (N = 64 queries, one chunk); K = 128 keys.
+      const uint64_t dq_a = sdesc_make(sdesc_lo(sK, C::KCHUNK), sdesc_hi(1024));
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_KV_FULL, 0, BF_MMA_KV));
+      tc_fence_after();
+      for (int it = 0; it <= nt && ok; ++it) {
+        if (it < nt) {
+          const int st = it % C::ST, b = it & 1;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_FULL + st), (it / C::ST) & 1, BF_MMA_Q))))
+            break;
+          tc_fence_after();
+          issue_t(tmem + C::TM_S + b * 64, sK, sQ + st * C::Q_TILE);
+          if (it >= 2) {  // dP^T's buffer holds dQ^T of tile it-2 until the drain has read it
+            if (!(ok = __all_sync(0xffffffffu,
+                                  mbar_wait(bars + 8 * (C::B_DQ_EMPTY + b), ((it >> 1) & 1) ^ 1, BF_MMA_DQE))))
+              break;
+            tc_fence_after();
+          }
+          issue_t(tmem + C::TM_DP + b * 64, sV, sdO + st * C::Q_TILE);
+          tc_commit_warp(bars + 8 * (C::B_S_FULL + b));
+        }
+        if (it > 0) {
+          const int pit = it - 1, pst = pit % C::ST, pb = pit & 1;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BF_MMA_P))))
+            break;
+          tc_fence_after();
+          issue_g(tmem + C::TM_DV, tmem + C::TM_S + pb * 64, sdO + pst * C::Q_TILE, pit > 0);
+          issue_g(tmem + C::TM_DK, tmem + C::TM_S + pb * 64 + 32, sQ + pst * C::Q_TILE, pit > 0);
+          tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + pst));
+          mma_ss_k128_mnmn(tmem + C::TM_DP + pb * 64, dq_a,
+                           sdesc_make(sdesc_lo(sDS + pb * C::DS_TILE, C::DS_TILE), sdesc_hi(1024)), IDESC_DQ, 0u);
+          tc_commit_warp(bars + 8 * (C::B_DQ_FULL + pb));
+        }
+      }
+      if (ok) tc_commit_warp(bars + 8 * C::B_DKV_FULL);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax gradient (thread = key row)
+    regs_inc<C::REGS_GRAD>();
+    const int sp = warp & 3;
+    const int r = sp * 32 + lane;
+    const int key = kt * C::BK + r;
+    const bool key_valid = key < N;
+    const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < nt; ++it) {
+      const int st = it % C::ST, b = it & 1;
+      const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
+      bool w = mbar_wait(bars + 8 * (C::B_S_FULL + b), (it >> 1) & 1, BF_SM_S);
+      w = w && mbar_wait(bars + 8 * (C::B_Q_FULL + st), (it / C::ST) & 1, BF_SM_Q);
+      if (!(ok = __all_sync(0xffffffffu, w))) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + C::TM_S + b * 64;
+      const uint32_t tP = tmem + lane_off + C::TM_DP + b * 64;
+      uint32_t sr[64], dr[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tP, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld_wait();
+      reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      const float* lse2 = sLSE + st * C::BQ;
+      const float* dd = sDD + st * C::BQ;
+      // masking: queries e < lim of this tile get P = 0 in this key row -- the
+      // causal mask (query q sees key j iff j <= q) and key rows past N
+      // (zero-filled K and V) -- so lim <= 0 means no masking
+      const int lim = !key_valid ? C::BQ : (CAUSAL ? key - qi * C::BQ : 0);
+      const bool mask = lim > 0;
+      uint8_t* ds_row = smem + C::OFF_DS + b * C::DS_TILE + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {  // 32 queries -> 16 packed columns of P^T and of dS^T
+        uint32_t pp[16], dsp[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = 32 * ch + 2 * c;
+          float p0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, -lse2[e]));
+          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, -lse2[e + 1]));
+          if (mask) {
+            if (e < lim) p0 = 0.f;
+            if (e + 1 < lim) p1 = 0.f;
+          }
+          const float ds0 = p0 * (__uint_as_float(dr[e]) - dd[e]);
+          const float ds1 = p1 * (__uint_as_float(dr[e + 1]) - dd[e + 1]);
+          pp[c] = pack_bf16(p0, p1);
+          dsp[c] = pack_bf16(ds0, ds1);
+        }
+        tmem_st16(tS + ch * 16, pp);
+        tmem_st16(tS + 32 + ch * 16, dsp);
+        // dS^T row r of the 128-byte-swizzled tile: 16-byte chunk j (queries
+        // 8j .. 8j+7) sits at chunk position j ^ (r % 8)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = 4 * ch + jj;
+          uint4 v;
+          v.x = dsp[4 * jj];
+          v.y = dsp[4 * jj + 1];
+          v.z = dsp[4 * jj + 2];
+          v.w = dsp[4 * jj + 3];
+          *reinterpret_cast<uint4*>(ds_row + ((j ^ (r & 7)) << 4)) = v;
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars + 8 * (C::B_P_FULL + b));
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_DKV_FULL, 0, BF_SM_DKV))) {
+      tc_fence_after();
+      const size_t base = (static_cast<size_t>(bh) * N + key) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tA = tmem + lane_off + (which ? C::TM_DK : C::TM_DV);
+        __nv_bfloat16* dst_row = (which ? dK : dV) + base;
+        const float mul = which ? scale : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tA + c * 32, a);
+          tmem_ld_wait();
+          reg_fence(a);
+          if (key_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 wv;
+              wv.x = pack_bf16(__uint_as_float(a[8 * v + 0]) * mul, __uint_as_float(a[8 * v + 1]) * mul);
+              wv.y = pack_bf16(__uint_as_float(a[8 * v + 2]) * mul, __uint_as_float(a[8 * v + 3]) * mul);
+              wv.z = pack_bf16(__uint_as_float(a[8 * v + 4]) * mul, __uint_as_float(a[8 * v + 5]) * mul);
+              wv.w = pack_bf16(__uint_as_float(a[8 * v + 6]) * mul, __uint_as_float(a[8 * v + 7]) * mul);
+              dst[v] = wv;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain (thread = column c of d)
+    regs_dec<C::REGS_DRAIN>();
+    const int sp = warp & 3;
+    const int c = sp * 32 + lane;
+    const bool active = c < D;  // d = 64: rows 64..127 of the product are V^T dS^T, not read
+    const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
+    const bool issuer = threadIdx.x == 256;
+    float* stg = reinterpret_cast<float*>(smem + C::OFF_DQ);
+    for (int it = 0; it < nt; ++it) {
+      const int b = it & 1, sb = it % C::NDQ;
+      const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
+      if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_DQ_FULL + b), (it >> 1) & 1, BF_DR_DQ))) break;
+      tc_fence_after();
+      // the staging buffer sb is free once the reduce issued NDQ tiles ago has read it
+      if (issuer) {
+        bulk_wait_read<C::NDQ - 1>();
+        mbar_arrive(bars + 8 * (C::B_STG_FREE + sb));
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (it / C::NDQ) & 1, BF_DR_FREE)))
+        break;
+      if (active) {  // 32 queries at a time: tensor memory -> registers -> [q][c] staging
+        float* t = stg + sb * (C::DQ_TILE / 4) + c;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::TM_DP + b * 64 + h * 32, v);
+          tmem_ld_wait();
+          reg_fence(v);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) t[(h * 32 + q) * D] = __uint_as_float(v[q]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bars + 8 * (C::B_DQ_EMPTY + b));
+      fence_proxy_async_smem();
+      mbar_arrive(bars + 8 * (C::B_STG_FULL + sb));
+      bool stored = true;
+      if (issuer) {
+        stored = mbar_wait(bars + 8 * (C::B_STG_FULL + sb), (it / C::NDQ) & 1, BF_DR_FULL);
+        if (stored) {
+          const int rows = min(C::BQ, N - qi * C::BQ);
+          bulk_reduce_add_f32(dQacc + (static_cast<size_t>(bh) * N + static_cast<size_t>(qi) * C::BQ) * D,
+                              sDQ + sb * C::DQ_TILE, static_cast<uint32_t>(rows * D * 4));
+          bulk_commit();
+        }
+      }
+      if (!__all_sync(0xffffffffu, stored)) break;
+    }
+    if (issuer) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ = bf16(scale * accumulator): eight elements per thread, 16-byte stores
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                                 __nv_bfloat16* __restrict__ dQ, long long n8,
+                                                                 float scale) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  uint4 w;
+  w.x = pack_bf16(a.x * scale, a.y * scale);
+  w.y = pack_bf16(a.z * scale, a.w * scale);
+  w.z = pack_bf16(b.x * scale, b.y * scale);
+  w.w = pack_bf16(b.z * scale, b.w * scale);
+  reinterpret_cast<uint4*>(dQ)[i] = w;
+}
+
+}  // namespace fa

@@ -382,6 +382,61 @@ __device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// K = 128, A and B both MN-major in shared memory (16 rows of 128 bytes =
+// +2048 B per K step for each): D^T-style products whose contraction runs
+// over the rows of both staged tiles.
+__device__ __forceinline__ void mma_ss_k128_mnmn(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 ax, bx;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %3, %3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 ax, %1, 128;\n\tadd.s64 bx, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 256;\n\tadd.s64 bx, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 384;\n\tadd.s64 bx, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 512;\n\tadd.s64 bx, %2, 512;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 640;\n\tadd.s64 bx, %2, 640;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 768;\n\tadd.s64 bx, %2, 768;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t"
+      "add.s64 ax, %1, 896;\n\tadd.s64 bx, %2, 896;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ax, bx, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// bulk (non-tensor) copies between shared and global memory
+// ---------------------------------------------------------------------------
+// Makes this thread's ordinary shared-memory stores visible to the async
+// proxy (the tensor core's operand reads, bulk copies) once a barrier orders
+// them before the consumer.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// global[dst .. dst+bytes) += shared[src .. src+bytes) as fp32, element-wise,
+// performed by the bulk-copy engine; both addresses 16-byte aligned, bytes a
+// multiple of 16.  Tracked by the issuing thread's bulk groups.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until every bulk group of this thread has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // 2-SM forms (cta_group::2): issued by the leader CTA of a pair; A and D rows
 // are split between the two CTAs (M/2 each), B's N columns likewise.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {

@@ -61,6 +61,8 @@ def load_library(build_if_missing: bool = True):
         lib.fa_bwd_workspace_bytes.restype = sz
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
         lib.fa_bwd.restype = i
+        lib.fa_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+        lib.fa_bwd_deterministic.restype = i
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
         lib.fa_bwd_noalloc.restype = i
         lib.fa_sync_status.argtypes = [vp]
@@ -106,17 +108,50 @@ def forward_kernel_name(d: int, causal: bool) -> str:
     return name.decode()
 
 
-def dkdv_kernel_name(d: int) -> str:
-    """Name of the dK/dV kernel `backward` launches for head size d
-    (fa_bwd_dkdv_kernel_name)."""
+def dkdv_kernel_name(d: int, deterministic: bool = False) -> str:
+    """Name of the kernel that computes dK and dV in `backward` for head size d
+    (fa_bwd_dkdv_kernel_name; the deterministic form runs fa_bwd_dkdv_kernel)."""
     name = load_library().fa_bwd_dkdv_kernel_name(int(d))
     if name is None:
         raise RuntimeError(f"no dK/dV kernel for d={d}")
-    return name.decode()
+    return "fa_bwd_dkdv_kernel" if deterministic else name.decode()
+
+
+def backward_kernel_names(d: int, deterministic: bool = False) -> tuple:
+    """The three kernels `backward` launches, in order (the phases that
+    set_backward_phase_events brackets)."""
+    if deterministic:
+        return ("fa_bwd_preprocess_kernel", "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel")
+    return ("fa_bwd_preprocess_kernel", dkdv_kernel_name(d), "fa_bwd_dq_convert_kernel")
+
+
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream_handle(device: torch.device):
+    """The current CUDA stream of `device` as a raw cudaStream_t."""
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(device.index))
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+class _NoSwitch:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+_NO_SWITCH = _NoSwitch()
+
+
+def _on(device: torch.device):
+    """Make `device` current for the call (the library works on the current
+    device); no switch when it already is."""
+    if device.index == torch.cuda.current_device():
+        return _NO_SWITCH
+    return torch.cuda.device(device)
 
 
 def _check_qkv(*ts: torch.Tensor):
@@ -145,7 +180,7 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     lib = load_library()
-    with torch.cuda.device(q.device):
+    with _on(q.device):
         rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
                         int(bool(causal)), _scale(scale, d), _stream_handle(q.device))
     if rc != FA_OK:
@@ -168,7 +203,7 @@ def forward_unfused(q, k, v, causal: bool = False, scale: float | None = None, w
     ws = torch.empty(nbytes, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    with torch.cuda.device(q.device):
+    with _on(q.device):
         rc = lib.fa_fwd_unfused(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, H, N, d,
                                 int(bool(causal)), _scale(scale, d), ws.data_ptr(), ws.numel(),
                                 _stream_handle(q.device))
@@ -182,8 +217,13 @@ def workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, workspace=None,
-             dq=None, dk=None, dv=None):
-    """dQ, dK, dV of sum(dO * O); inputs as produced by forward()."""
+             dq=None, dk=None, dv=None, deterministic: bool = False):
+    """dQ, dK, dV of sum(dO * O); inputs as produced by forward().
+
+    Default (fa_bwd): one kernel forms all five products per tile and adds dQ
+    partial sums into an fp32 accumulator, so dQ's last bits can vary between
+    runs.  deterministic=True (fa_bwd_deterministic): a separate dQ kernel,
+    bit-reproducible, slower."""
     _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
@@ -194,19 +234,20 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
-    with torch.cuda.device(q.device):
-        rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
-                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)),
-                        _scale(scale, d), ws.data_ptr(), ws.numel(), _stream_handle(q.device))
+    fn = lib.fa_bwd_deterministic if deterministic else lib.fa_bwd
+    with _on(q.device):
+        rc = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)),
+                _scale(scale, d), ws.data_ptr(), ws.numel(), _stream_handle(q.device))
     if rc != FA_OK:
-        raise FaError(rc, "fa_bwd")
+        raise FaError(rc, "fa_bwd_deterministic" if deterministic else "fa_bwd")
     return dq, dk, dv
 
 
 def backward_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, dq=None, dk=None,
                      dv=None):
-    """backward() without a workspace: the library's fixed 4 MiB device array
-    holds D (B*H*N <= NOALLOC_MAX_ROWS).  For callers that cannot allocate
+    """backward(deterministic=True) without a workspace: the library's fixed
+    4 MiB device array holds D (B*H*N <= NOALLOC_MAX_ROWS).  For callers that cannot allocate
     device memory; pass preallocated dq/dk/dv to allocate nothing at all.
     Calls that overlap on the GPU share the array and race."""
     _check_qkv(q, k, v, o, do)
@@ -217,7 +258,7 @@ def backward_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | N
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     lib = load_library()
-    with torch.cuda.device(q.device):
+    with _on(q.device):
         rc = lib.fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                 lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
                                 int(bool(causal)), _scale(scale, d), _stream_handle(q.device))
@@ -233,8 +274,9 @@ def sync_status(device=None) -> int:
 
 
 def set_backward_phase_events(events=None) -> None:
-    """Record four torch.cuda.Event objects around fa_bwd's kernels (D pass,
-    dK/dV, dQ); None stops.  The events must outlive their use."""
+    """Record four torch.cuda.Event objects around the backward's three
+    kernels (backward_kernel_names); None stops.  The events must outlive
+    their use."""
     lib = load_library()
     if events is None:
         lib.fa_bwd_set_phase_events(None, None, None, None)
@@ -243,6 +285,11 @@ def set_backward_phase_events(events=None) -> None:
             if e.cuda_event == 0:
                 e.record()
         lib.fa_bwd_set_phase_events(*[ctypes.c_void_p(e.cuda_event) for e in events])
+
+
+def last_cuda_error() -> int:
+    """The cudaError_t behind the last FA_ERR_LAUNCH (fa_last_cuda_error)."""
+    return int(load_library().fa_last_cuda_error())
 
 
 def last_error_word() -> int:

@@ -25,7 +25,8 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == {"fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_sync_status", "fa_last_error_word",
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
                           "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name",
-                          "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes", "fa_bwd_dkdv_kernel_name"}
+                          "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes", "fa_bwd_dkdv_kernel_name",
+                          "fa_bwd_deterministic"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:
@@ -42,8 +43,10 @@ def test_status_strings(lib):
 
 
 def test_workspace_bytes(lib):
-    assert lib.fa_bwd_workspace_bytes(2, 16, 4096, 128) == 2 * 16 * 4096 * 4
-    assert lib.fa_bwd_workspace_bytes(8, 12, 1000, 64) == ((8 * 12 * 1000 * 4 + 255) // 256) * 256
+    # D (fp32 per row, padded to 256 bytes), then the fp32 dQ accumulator
+    assert lib.fa_bwd_workspace_bytes(2, 16, 4096, 128) == 2 * 16 * 4096 * 4 + 2 * 16 * 4096 * 128 * 4
+    assert lib.fa_bwd_workspace_bytes(8, 12, 1000, 64) == (((8 * 12 * 1000 * 4 + 255) // 256) * 256
+                                                           + 8 * 12 * 1000 * 64 * 4)
     assert lib.fa_bwd_workspace_bytes(1, 1, 0, 64) == 0
     assert lib.fa_bwd_workspace_bytes(1, 1, 16, 96) == 0
 
@@ -134,19 +137,39 @@ def test_unfused_rejects_bad_arguments(lib):
         assert _unf(lib) == EDEV
 
 
-def test_dkdv_kernel_name_follows_the_settings(monkeypatch):
+def test_dkdv_kernel_name():
     # pure host logic: no device needed
-    monkeypatch.delenv("FA_BWD_PAIR", raising=False)
-    monkeypatch.delenv("FA_BWD_PERSIST", raising=False)
-    assert fa.dkdv_kernel_name(128) == "fa_bwd_dkdv_kernel"
-    assert fa.dkdv_kernel_name(64) == "fa_bwd_dkdv_kernel"
-    monkeypatch.setenv("FA_BWD_PERSIST", "1")
-    assert fa.dkdv_kernel_name(128) == "fa_bwd_dkdv_persistent_kernel"
-    monkeypatch.setenv("FA_BWD_PAIR", "1")
-    assert fa.dkdv_kernel_name(128) == "fa_bwd_dkdv_2sm_kernel"
-    assert fa.dkdv_kernel_name(64) == "fa_bwd_dkdv_persistent_kernel"
+    assert fa.dkdv_kernel_name(128) == "fa_bwd_fused_kernel"
+    assert fa.dkdv_kernel_name(64) == "fa_bwd_fused_kernel"
+    assert fa.dkdv_kernel_name(128, deterministic=True) == "fa_bwd_dkdv_kernel"
+    assert fa.backward_kernel_names(64) == ("fa_bwd_preprocess_kernel", "fa_bwd_fused_kernel",
+                                            "fa_bwd_dq_convert_kernel")
+    assert fa.backward_kernel_names(128, True) == ("fa_bwd_preprocess_kernel", "fa_bwd_dkdv_kernel",
+                                                   "fa_bwd_dq_kernel")
     with pytest.raises(RuntimeError):
         fa.dkdv_kernel_name(96)
+
+
+def _bwd_det(lib, ws=20 * A, ws_bytes=None, B=1, H=1, N=128, d=64, **ptrs):
+    p = dict(q=A, k=2 * A, v=3 * A, o=4 * A, do=5 * A, lse=6 * A, dq=7 * A, dk=8 * A, dv=9 * A)
+    p.update(ptrs)
+    nb = ((B * H * N * 4 + 255) // 256) * 256 if ws_bytes is None else ws_bytes
+    return lib.fa_bwd_deterministic(p["q"], p["k"], p["v"], p["o"], p["do"], p["lse"], p["dq"], p["dk"], p["dv"],
+                                    B, H, N, d, 1, 0.0, ws, nb, None)
+
+
+def test_deterministic_backward_needs_only_the_d_part(lib):
+    """fa_bwd_deterministic takes the same arguments as fa_bwd but uses only
+    the D part of the workspace; fa_bwd needs D and the dQ accumulator."""
+    d_bytes = ((128 * 4 + 255) // 256) * 256
+    assert _bwd_det(lib, ws_bytes=d_bytes - 16) == EWS
+    assert _bwd(lib, ws_bytes=d_bytes) == EWS
+    assert _bwd_det(lib, N=0) == EINVAL
+    assert _bwd_det(lib, dk=8 * A + 4) == EALIGN
+    assert _bwd_det(lib, dq=A) == EINVAL
+    if not torch.cuda.is_available():
+        assert _bwd_det(lib, ws_bytes=d_bytes) == EDEV   # valid arguments: stops at the device check
+        assert _bwd(lib) == EDEV
 
 
 def test_selftest_rejects_bad_limit(lib):

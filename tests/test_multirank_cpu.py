@@ -58,3 +58,42 @@ def test_whole_job_throughput_counts_every_rank():
     assert bench.whole_job_tflops(2, 1e12, 10, 10.0) == pytest.approx(2000.0)
     assert bench.whole_job_tflops(1, 1e12, 10, 10.0) == pytest.approx(1000.0)
     assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def _run_bench(args, env_extra=None, timeout=600):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env.update(env_extra or {})
+    r = subprocess.run([sys.executable, "bench.py", *args], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=timeout)
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    return r, lines
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` with no launcher starts two ranks through
+    torch.distributed.run (rendezvous on 127.0.0.1).  The reference arm runs
+    on the host cores, so the launcher is exercised here without a GPU: rank 0
+    prints the one line, with n_gpus = 2; rank 1 exits without work."""
+    r, lines = _run_bench(["--gpus", "2", "--impl", "reference", "--steps", "1", "--warmup", "0"])
+    assert r.returncode == 0, r.stderr[-3000:]
+    assert len(lines) == 1, r.stdout
+    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_gpus_flag_and_world_size_must_agree():
+    """A rank whose WORLD_SIZE differs from --gpus refuses to time anything."""
+    r, lines = _run_bench(["--gpus", "2", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                          env_extra={"WORLD_SIZE": "1", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode == 2 and not lines
+    assert "WORLD_SIZE=1" in r.stderr
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the refusal when GPUs are missing")
+def test_gpu_arm_refuses_more_ranks_than_devices():
+    r, lines = _run_bench(["--gpus", "2", "--steps", "1", "--warmup", "0"])
+    assert r.returncode == 2 and not lines
+    assert "visible CUDA devices" in r.stderr

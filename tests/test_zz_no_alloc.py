@@ -1,11 +1,14 @@
 """fa_bwd_noalloc: the backward for callers that cannot allocate device memory
 (a plugin given only its input and output buffers, code under a memory pool
-that must not grow).  Its D vector lives in the library's fixed device array.
+that must not grow).  Its D vector lives in the library's fixed device array,
+and it runs the deterministic form of the backward, whose only scratch is D.
 
-Checked through the C ABI against fa_bwd (the workspace version) on two calls
-in a row with different shapes, so stale contents of the shared array would
-show.  This file sorts last so that a run stopping at the first failure has
-already run every other test.
+Checked through the C ABI on two calls in a row with different shapes (stale
+contents of the shared array would show): bit-identical to
+fa_bwd_deterministic given a workspace, and within the gradient tolerance of
+fa_bwd.  One more call fills the array exactly (B*H*N = FA_NOALLOC_MAX_ROWS).
+This file sorts last so that a run stopping at the first failure has already
+run every other test.
 """
 from __future__ import annotations
 
@@ -16,7 +19,7 @@ import torch
 
 from io_aware_tiled_b200 import fa
 from io_aware_tiled_b200.inputs import attention_inputs
-from tests.parity import GRAD_REL_FROB, f64, rel_frob
+from tests.parity import GRAD_REL_FROB, assert_same_up_to_summation_order, f64, rel_frob
 
 pytestmark = pytest.mark.gpu
 
@@ -38,13 +41,35 @@ def test_noalloc_backward_matches_workspace_backward():
     for (B, H, N, d, causal) in [(2, 3, 1000, 128, True), (1, 4, 777, 64, False)]:
         q, k, v, do = (t.to(dev) for t in attention_inputs(B, H, N, d, seed=N))
         o, lse = fa.forward(q, k, v, causal)
-        ref = fa.backward(q, k, v, o, do, lse, causal)
+        det = fa.backward(q, k, v, o, do, lse, causal, deterministic=True)
+        fused = fa.backward(q, k, v, o, do, lse, causal)
         rc, got = _call_noalloc(lib, q, k, v, o, do, lse, causal)
         assert rc == fa.FA_OK, fa.status_string(rc)
         assert fa.sync_status(dev) == fa.FA_OK
-        for name, g, r in zip(("dq", "dk", "dv"), got, ref):
-            err = rel_frob(f64(g), f64(r))
+        for name, g, r, f in zip(("dq", "dk", "dv"), got, det, fused):
+            assert torch.equal(g, r), (B, H, N, d, causal, name)
+            err = rel_frob(f64(g), f64(f))
             assert err <= GRAD_REL_FROB, (B, H, N, d, causal, name, err)
+        assert_same_up_to_summation_order(got[0], fused[0], f"dQ {B, H, N, d} causal={causal}")
+
+
+def test_noalloc_fills_its_array_exactly():
+    """B*H*N = FA_NOALLOC_MAX_ROWS: the largest size the array takes; every
+    row of D is used.  Still bit-identical to fa_bwd_deterministic."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dev = torch.device("cuda", 0)
+    lib = fa.load_library()
+    B, H, N, d = 2, 32, 16384, 64
+    assert B * H * N == fa.NOALLOC_MAX_ROWS
+    q, k, v, do = (t.to(dev) for t in attention_inputs(B, H, N, d, seed=3))
+    o, lse = fa.forward(q, k, v, True)
+    det = fa.backward(q, k, v, o, do, lse, True, deterministic=True)
+    rc, got = _call_noalloc(lib, q, k, v, o, do, lse, True)
+    assert rc == fa.FA_OK, fa.status_string(rc)
+    assert fa.sync_status(dev) == fa.FA_OK
+    for name, g, r in zip(("dq", "dk", "dv"), got, det):
+        assert torch.equal(g, r), name
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
