@@ -185,7 +185,49 @@ def oracle_sample_run(N=4096, d=128, causal=False, heads=1, seed=0):
     return dt, f + b
 
 
-def cpu_baseline(target_s=12.0):
+def oracle_workload_samples():
+    """The oracle on a bounded sample of every named workload (about 15 s in
+    all): the single-head workload in full, on all cores and on one core; one
+    head of the headline forward (both masks); one head of the training and
+    long-sequence workloads (fwd+bwd, causal); the ragged d=64 workload in full
+    (fwd+bwd, both masks).  TFLOP/s by the conventional count of the sample."""
+    import oracle
+    from io_aware_tiled_b200.configs import WORKLOADS
+    from io_aware_tiled_b200.inputs import attention_inputs
+    out = []
+    plan = [("pr1_b1h1n256d64", False, "fwd", None), ("pr1_b1h1n256d64", False, "fwd", 1),
+            ("fwd_b2h16n4096d128", False, "fwd", None), ("fwd_b2h16n4096d128", True, "fwd", None),
+            ("train_b4h32n2048d128", True, "fwd+bwd", None), ("long_b1h16n16384d128", True, "fwd+bwd", None),
+            ("ragged_b8h12n1000d64", False, "fwd+bwd", None), ("ragged_b8h12n1000d64", True, "fwd+bwd", None)]
+    all_threads = oracle.num_threads()
+    for name, causal, pas, threads in plan:
+        w = WORKLOADS[name]
+        heads = w.B * w.H if name in ("pr1_b1h1n256d64", "ragged_b8h12n1000d64") else 1
+        B, H = (w.B, w.H) if heads == w.B * w.H else (1, 1)
+        q, k, v, do = (t.double().numpy() if t is not None else None
+                       for t in attention_inputs(B, H, w.N, w.d, seed=w.seed, sigma_qk=w.sigma_qk,
+                                                 with_do=pas != "fwd"))
+        if threads:
+            oracle.set_num_threads(threads)
+        try:
+            t0 = time.perf_counter()
+            if pas == "fwd":
+                oracle.forward(q, k, v, causal, w.scale)
+            else:
+                oracle.backward(q, k, v, do, causal, w.scale)
+            dt = time.perf_counter() - t0
+        finally:
+            if threads:
+                oracle.set_num_threads(all_threads)
+        f, b = _flops(B, H, w.N, w.d, causal)
+        fl = f + (b if pas != "fwd" else 0.0)
+        out.append({"workload": name, "causal": causal, "pass": pas,
+                    "sample": "full workload" if heads == w.B * w.H else "one head",
+                    "threads": threads or all_threads, "seconds": dt, "tflops": fl / dt / 1e12})
+    return out
+
+
+def cpu_baseline(target_s=6.0):
     import oracle
     total_t, total_f, reps = 0.0, 0.0, 0
     while total_t < target_s and reps < 8:
@@ -195,7 +237,8 @@ def cpu_baseline(target_s=12.0):
         reps += 1
     return {"value": total_f / total_t / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{reps} x one head (B=1,H=1,N=4096,d=128) fwd+bwd non-causal, fp64, {total_t:.1f} s",
-            "host_cpu_count": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
+            "host_cpu_count": os.cpu_count(), "affinity": len(os.sched_getaffinity(0)),
+            "workloads": oracle_workload_samples()}
 
 
 def run_reference(args, rank, world):
@@ -610,7 +653,24 @@ def time_workloads(steps: int, warmup: int, dev, reduce_max=lambda x: x, skip=()
                         line["gbs_best"] = io_bytes / (best * 1e-3) / 1e9
                     lines.append(line)
                 if small:
-                    # latency-bound: the same call replayed from a CUDA graph
+                    # latency-bound: `steps` eager calls back to back between two
+                    # events (the host enqueues the next call while the GPU runs
+                    # the current one), per call
+                    for _ in range(warmup):
+                        fn()
+                    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    torch.cuda.synchronize()
+                    a_.record()
+                    for _ in range(steps):
+                        fn()
+                    b_.record()
+                    torch.cuda.synchronize()
+                    per = reduce_max(a_.elapsed_time(b_) / steps)
+                    lines.append({"workload": w.name, "causal": causal, "pass": name, "launch": "eager, back to back",
+                                  "mean_us": per * 1e3, "tflops_mean": flops / (per * 1e-3) / 1e12,
+                                  "gbs_mean": io_bytes / (per * 1e-3) / 1e9 if name == "fwd" else None,
+                                  "l2": "warm (no flush)", "steps": steps, "warmup": warmup})
+                    # the same call replayed from a CUDA graph
                     # (no host-side work between the events)
                     fn()
                     torch.cuda.synchronize()

@@ -52,7 +52,7 @@
 
 namespace fa {
 
-template <int D, int ST_ = ((D == 128) ? 2 : 4), int NDQ_ = 2>
+template <int D, int ST_ = ((D == 128) ? 3 : 4), int NDQ_ = ((D == 128) ? 1 : 2)>
 struct FusedCfg {
   static constexpr int BK = 128;                      // keys per CTA (MMA M of S^T, dP^T, dV, dK)
   static constexpr int BQ = 64;                       // queries per tile
@@ -110,7 +110,7 @@ __device__ __forceinline__ int fused_query_tile(int it, int i0, int nt, int kt) 
   return q;
 }
 
-template <int D, bool CAUSAL, int ST_ = ((D == 128) ? 2 : 4), int NDQ_ = 2>
+template <int D, bool CAUSAL, int ST_ = ((D == 128) ? 3 : 4), int NDQ_ = ((D == 128) ? 1 : 2)>
 __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
     fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
