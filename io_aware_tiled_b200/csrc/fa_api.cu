@@ -215,7 +215,7 @@ struct RangeEntry {
   uintptr_t lo = 0, hi = 0;
   int dev = -1;
 };
-constexpr int kRangeCache = 256;
+constexpr int kRangeCache = 64;
 RangeEntry g_ranges[kRangeCache];
 int g_ranges_next = 0;
 std::mutex g_ranges_mu;
@@ -241,8 +241,10 @@ bool is_device_ptr(const void* p, size_t bytes = 1) {
   const uintptr_t lo = reinterpret_cast<uintptr_t>(p), hi = lo + (bytes ? bytes : 1);
   {
     std::lock_guard<std::mutex> lock(g_ranges_mu);
-    for (const RangeEntry& e : g_ranges)
+    for (int i = 1; i <= kRangeCache; ++i) {  // most recently added first
+      const RangeEntry& e = g_ranges[(g_ranges_next - i + kRangeCache) % kRangeCache];
       if (e.dev == dev && lo >= e.lo && hi <= e.hi) return true;
+    }
   }
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
@@ -535,6 +537,11 @@ static int bwd_launch(const void* Q, const void* K, const void* V, const void* O
   if (!fused && (!make_map(&mq128, Q, BH, N, d, 128) || !make_map(&mdo128, dO, BH, N, d, 128) ||
                  !make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64)))
     return encode_failed();
+  // the fused kernel's query tiles: boxes of its BQ rows
+  CUtensorMap mqf, mdof;
+  const int fused_bq = d == 64 ? fa::FusedCfg<64>::BQ : fa::FusedCfg<128>::BQ;
+  if (fused && (!make_map(&mqf, Q, BH, N, d, fused_bq) || !make_map(&mdof, dO, BH, N, d, fused_bq)))
+    return encode_failed();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   clear_stale_error();
   float* Dvec = static_cast<float*>(workspace);
@@ -563,8 +570,8 @@ static int bwd_launch(const void* Q, const void* K, const void* V, const void* O
     if (fused) {
       fa::fa_bwd_preprocess_kernel<64, true><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows, dqacc);
       mark(1);
-      if (causal) fa::fa_bwd_fused_kernel<64, true><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
-      else fa::fa_bwd_fused_kernel<64, false><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      if (causal) fa::fa_bwd_fused_kernel<64, true><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      else fa::fa_bwd_fused_kernel<64, false><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
       mark(2);
       fa::fa_bwd_dq_convert_kernel<<<grid_cvt, 256, 0, s>>>(dqacc, dq, rows * d / 8, sc);
     } else {
@@ -580,8 +587,8 @@ static int bwd_launch(const void* Q, const void* K, const void* V, const void* O
     if (fused) {
       fa::fa_bwd_preprocess_kernel<128, true><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows, dqacc);
       mark(1);
-      if (causal) fa::fa_bwd_fused_kernel<128, true><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
-      else fa::fa_bwd_fused_kernel<128, false><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mq64, mk128, mv128, mdo64, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      if (causal) fa::fa_bwd_fused_kernel<128, true><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      else fa::fa_bwd_fused_kernel<128, false><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
       mark(2);
       fa::fa_bwd_dq_convert_kernel<<<grid_cvt, 256, 0, s>>>(dqacc, dq, rows * d / 8, sc);
     } else {
