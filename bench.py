@@ -753,7 +753,8 @@ def run_tile_sweep(steps: int, warmup: int):
                 f, _ = _flops(B, H, N, d, causal)
                 bq = 128  # query rows per softmax warpgroup / TMEM lane block
                 q_tiles_per_sm = tq // bq
-                smem = q_tiles_per_sm * bq * d * 2 + st * 2 * (tk if name == "one-SM" else tk // 2) * d * 2
+                q_bufs = 2 if (name == "one-SM" and d == 64) else 1  # d = 64 keeps two Q pairs
+                smem = q_bufs * q_tiles_per_sm * bq * d * 2 + st * 2 * (tk if name == "one-SM" else tk // 2) * d * 2
                 tmem_cols = ns * tk + q_tiles_per_sm * d if name == "one-SM" else ns * tk + d
                 pages_sram = bq * d * 2 + 2 * tk * d * 2 + bq * tk * 2 + bq * d * 2 + bq * 8
                 print(json.dumps({

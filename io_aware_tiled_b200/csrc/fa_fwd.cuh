@@ -19,7 +19,9 @@
 //   * Three warpgroups: the control warpgroup gives registers back
 //     (setmaxnreg) to the two softmax warpgroups, which hold a full S row each.
 //   * Warp 0 issues TMA loads: Q pair once per unit, K_j and V_j through
-//     separate rings of ST stages (128 keys x d, 128-byte swizzle).
+//     separate rings of ST stages (128 keys x d, 128-byte swizzle).  At
+//     d = 64 shared memory holds two Q pairs, so the next unit's Q arrives
+//     while the current unit still runs (NQB buffers).
 //   * Warp 1 issues tcgen05.mma from one thread: S_t = Q_t K_j^T (M=128,
 //     N=128, K=d, both operands K-major in shared memory) into tensor memory,
 //     and O_t += P_t V_j (M=128, N=d, K=128) with P_t read from TENSOR MEMORY
@@ -50,14 +52,16 @@ struct FwdCfg {
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int KV_TILE = BN * D * 2;
   static constexpr int ST = ((D == 128) ? 2 : 4) * R;  // K and V ring depth (same bytes for either BN)
+  static constexpr int NQB = (D == 64) ? 2 : 1;  // Q-pair buffers (the next unit's Q loads early)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_K = OFF_Q + NQB * 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + ST * KV_TILE;
   static constexpr int OFF_BAR = OFF_V + ST * KV_TILE;
   // barrier indices
-  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
-  static constexpr int B_K_FULL = 2, B_K_EMPTY = 2 + ST, B_V_FULL = 2 + 2 * ST, B_V_EMPTY = 2 + 3 * ST;
-  static constexpr int B_S_FULL = 2 + 4 * ST, B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2,
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = NQB;
+  static constexpr int B_K_FULL = 2 * NQB, B_K_EMPTY = 2 * NQB + ST, B_V_FULL = 2 * NQB + 2 * ST,
+                       B_V_EMPTY = 2 * NQB + 3 * ST;
+  static constexpr int B_S_FULL = 2 * NQB + 4 * ST, B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2,
                        B_O_EMPTY = B_O_FULL + 2;
   static constexpr int NUM_BARS = B_O_EMPTY + 2;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
@@ -111,8 +115,10 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + 8 * C::B_Q_FULL, 1);
-    mbar_init(bars + 8 * C::B_Q_EMPTY, 1);
+    for (int qb = 0; qb < C::NQB; ++qb) {
+      mbar_init(bars + 8 * (C::B_Q_FULL + qb), 1);
+      mbar_init(bars + 8 * (C::B_Q_EMPTY + qb), 1);
+    }
     for (int s = 0; s < C::ST; ++s) {
       mbar_init(bars + 8 * (C::B_K_FULL + s), 1);
       mbar_init(bars + 8 * (C::B_K_EMPTY + s), 1);
@@ -158,12 +164,13 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
         const int nk1 = CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT;
-        if (!mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it & 1) ^ 1, FW_PROD_Q)) break;
+        const int qb = q_it % C::NQB;
+        if (!mbar_wait(bars + 8 * (C::B_Q_EMPTY + qb), ((q_it / C::NQB) & 1) ^ 1, FW_PROD_Q)) break;
         ++q_it;
-        mbar_arrive_expect_tx(bars + 8 * C::B_Q_FULL, 2 * C::Q_TILE);
+        mbar_arrive_expect_tx(bars + 8 * (C::B_Q_FULL + qb), 2 * C::Q_TILE);
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::CH; ++c)
-            tma_load_3d(sQ + t * C::Q_TILE + c * C::CHUNK, &tmQ, bars + 8 * C::B_Q_FULL, c * 64,
+            tma_load_3d(sQ + (qb * 2 + t) * C::Q_TILE + c * C::CHUNK, &tmQ, bars + 8 * (C::B_Q_FULL + qb), c * 64,
                         (2 * qp + t) * C::BM, bh);
         bool ok = true;
         for (int j = 0; j < nk1; ++j, ++kv_it) {
@@ -216,7 +223,9 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
         (void)bh;
         const int nk0 = CAUSAL ? min((2 * qp + 1) * C::R, NKT) : NKT;
         const int nk1 = CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT;
-        bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_FULL, q_it & 1, FW_MMA_Q));
+        const int qb = q_it % C::NQB;
+        const uint32_t sQb = sQ + qb * 2 * C::Q_TILE;
+        bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_FULL + qb), (q_it / C::NQB) & 1, FW_MMA_Q));
         ++q_it;
         if (!ok) break;
         tc_fence_after();
@@ -224,9 +233,9 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           const int s = kv_it % C::ST;
           if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_K_FULL + s), (kv_it / C::ST) & 1, FW_MMA_K))) break;
           tc_fence_after();
-          issue_s(tmem + C::TM_S0, sQ, sK + s * C::KV_TILE);
+          issue_s(tmem + C::TM_S0, sQb, sK + s * C::KV_TILE);
           tc_commit_warp(bars + 8 * (C::B_S_FULL + 0));
-          issue_s(tmem + C::TM_S1, sQ + C::Q_TILE, sK + s * C::KV_TILE);
+          issue_s(tmem + C::TM_S1, sQb + C::Q_TILE, sK + s * C::KV_TILE);
           tc_commit_warp(bars + 8 * (C::B_S_FULL + 1));
           tc_commit_warp(bars + 8 * (C::B_K_EMPTY + s));
         }
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           }
           if (more) {
             if (j + 1 < nk0) {
-              issue_s(tmem + C::TM_S0, sQ, sK + sn * C::KV_TILE);
+              issue_s(tmem + C::TM_S0, sQb, sK + sn * C::KV_TILE);
               tc_commit_warp(bars + 8 * (C::B_S_FULL + 0));
             }
           }
@@ -262,18 +271,20 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           tc_commit_warp(bars + 8 * (C::B_V_EMPTY + s));
           if (j == nk1 - 1) tc_commit_warp(bars + 8 * (C::B_O_FULL + 1));
           if (more) {
-            issue_s(tmem + C::TM_S1, sQ + C::Q_TILE, sK + sn * C::KV_TILE);
+            issue_s(tmem + C::TM_S1, sQb + C::Q_TILE, sK + sn * C::KV_TILE);
             tc_commit_warp(bars + 8 * (C::B_S_FULL + 1));
             tc_commit_warp(bars + 8 * (C::B_K_EMPTY + sn));
           }
         }
         if (!ok) break;
-        tc_commit_warp(bars + 8 * C::B_Q_EMPTY);
+        tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));
         kv_it += nk1;
       }
       // The last unit's Q_EMPTY arrival is the last one this thread's commits
       // make; wait for it so no arrival lands after the CTA has exited.
-      if (q_it > 0) (void)__all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_Q_EMPTY, (q_it - 1) & 1, FW_MMA_Q));
+      if (q_it > 0)
+        (void)__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_EMPTY + (q_it - 1) % C::NQB),
+                                                ((q_it - 1) / C::NQB) & 1, FW_MMA_Q));
     }
     }
     // teardown (each branch has its own, so the register regions never merge)
