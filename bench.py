@@ -297,22 +297,18 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # DRAM traffic from ncu
 # ---------------------------------------------------------------------------
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of each kernel,
-# captured with `python bench.py --ncu-case fwd|bwd` (B=4, H=16, N=4096,
-# d=128, non-causal: 64 heads) and divided by the 64 heads; the summaries sit
-# in profiles/.  Each kernel reads its inputs once per head, so the traffic of
-# the bench's 32-head launch is the per-head figure x 32.  Each entry keeps the
+# captured with `python bench.py --ncu-case fwd|bwd --ncu-batch B` and divided
+# by the B*16 heads; the summaries sit in profiles/.  Each kernel reads its
+# inputs once per head, so the traffic of the bench's 32-head launch is the
+# per-head figure x 32.  Each entry keeps the
 # sha256 of the sources the kernel is compiled from at capture time: once they
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
-    "fa_fwd_2sm_kernel": {"bytes_per_head": (201.415168e6 + 51.269120e6) / 64,
-                          "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "94c61c24f4f62b4c19a61f4d9c82f9dda1b8a2b78f43214dd4ac47f54b83e257"},
-    "fa_bwd_dkdv_kernel": {"bytes_per_head": (270.758144e6 + 103.693824e6) / 64,
-                           "sources": ("fa_bwd.cuh", "fa_device.cuh"),
-                           "sha256": "105e14ddf5f946b5e6b5ba46e955de295b09f20301f310c4494f0d2e4e6f0234"},
-    "fa_bwd_dq_kernel": {"bytes_per_head": (270.868736e6 + 52.507392e6) / 64,
-                         "sources": ("fa_bwd.cuh", "fa_device.cuh"),
-                         "sha256": "105e14ddf5f946b5e6b5ba46e955de295b09f20301f310c4494f0d2e4e6f0234"},
+    # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
+    # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
+    "fa_bwd_fused_kernel": {"bytes_per_head": (202.540544e6 + 86.772480e6) / 32,
+                            "sources": ("fa_bwd_fused.cuh", "fa_device.cuh"),
+                            "sha256": "8dab14cec0ee2fc62a21f534d140f5bc794e235b6ef798c6fa0e0184840fd84d"},
 }
 
 
@@ -460,9 +456,13 @@ def run_ours(args, rank, world, local_rank):
 
     from io_aware_tiled_b200.host_pipeline import forward_backward_host
 
+    ws_host = torch.empty(fa.host_workspace_bytes(B, H, N, d, 8), dtype=torch.uint8, device=dev)
+
     def e2e_pipelined():
-        # heads in groups through three streams: copies in, kernels, copies out
-        forward_backward_host(hq, hk, hv, hdo, False, out=(ho, hl, hdq, hdk, hdv), device=dev)
+        # fa_fwd_bwd_host: heads in groups through the library's three streams
+        # (copies in, kernels, copies out)
+        forward_backward_host(hq, hk, hv, hdo, False, groups=8, out=(ho, hl, hdq, hdk, hdv), workspace=ws_host,
+                              device=dev)
 
     e2e_steps = max(3, args.steps // 4)
     for _ in range(2):
@@ -563,7 +563,7 @@ def run_ours(args, rank, world, local_rank):
             # inputs, runs the kernels, then copies all outputs back
             "e2e": {"value": world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps,
-                    "api": "io_aware_tiled_b200.host_pipeline.forward_backward_host",
+                    "api": "fa_fwd_bwd_host (C ABI), called through io_aware_tiled_b200.fa.forward_backward_host",
                     "serial_value": world * step_flops * e2e_steps / (e2e_serial_ms * 1e-3) / 1e12,
                     "serial_ms_per_step": e2e_serial_ms / e2e_steps},
             "workloads": wlines,

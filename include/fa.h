@@ -116,6 +116,35 @@ int fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void
                          float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward and backward from host memory to host memory, for callers whose
+ * data lives on the host: the pages' problem statement run end to end, with
+ * the PCIe copies overlapped with the kernels.
+ * In (host or device memory, page-locked host memory for the copies to
+ * overlap): Q, K, V, dO [B,H,N,d] bf16.
+ * Out (same kinds of memory): O [B,H,N,d] bf16, LSE [B,H,N] fp32, dQ, dK, dV
+ * [B,H,N,d] bf16 -- what fa_fwd followed by fa_bwd produce.
+ * The B*H heads go in `groups` (1 .. B*H; more are clamped) consecutive groups
+ * of ceil(B*H / groups) heads.  Three of the library's own streams, created at
+ * the first call on each device and kept, carry the copies of group c to the
+ * device, fa_fwd + fa_bwd on group c-1 and the copies of group c-2 back, so
+ * both copy directions and the kernels run at the same time.
+ * workspace: caller-owned device memory of at least
+ * fa_fwd_bwd_host_workspace_bytes(B, H, N, d, groups) bytes (three slots, each
+ * holding one group's inputs, outputs and backward workspace), 16-byte
+ * aligned.  The call allocates nothing.
+ * stream: the pipeline starts after the work already queued on `stream`, and
+ * `stream` waits for the whole pipeline: once it synchronizes, the outputs
+ * are in host memory.  Calls from several threads are queued one after
+ * another.  Returns FA_OK or an fa_status code; validation errors return
+ * before anything is queued; an error from a group's kernels returns with
+ * earlier groups already queued (outputs then undefined).
+ */
+size_t fa_fwd_bwd_host_workspace_bytes(int B, int H, int N, int d, int groups);
+int fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const void* dO, void* O, float* LSE, void* dQ,
+                    void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, int groups,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_bwd for callers that cannot allocate device memory -- for example a
  * plugin whose host runtime hands it only its input and output buffers, or
  * code running under a memory pool that must not grow.  The paper has no

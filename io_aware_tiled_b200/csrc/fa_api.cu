@@ -752,3 +752,162 @@ extern "C" int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const
   return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, scratch,
                     static_cast<size_t>(FA_NOALLOC_MAX_ROWS) * sizeof(float), stream, false);
 }
+
+// ---------------------------------------------------------------------------
+// fa_fwd_bwd_host: forward + backward from host memory to host memory, the
+// PCIe copies overlapped with the kernels
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kHostSlots = 3;  // copy-in of group c, kernels of c-1 and copy-out of c-2 run at once
+
+// The library's own streams and events for the pipeline, one set per device,
+// created at the first call on that device and kept until the process exits.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t s_in = nullptr, s_run = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t ev_in[kHostSlots] = {}, ev_run[kHostSlots] = {}, ev_out[kHostSlots] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;  // held for a whole call's enqueue: the streams and events are shared
+
+bool host_pipe_ready(HostPipe& p) {
+  if (p.ready) return true;
+  bool ok = cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.s_run, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.done, cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; i < kHostSlots && ok; ++i)
+    ok = cudaEventCreateWithFlags(&p.ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p.ev_run[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p.ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+  p.ready = ok;
+  return ok;
+}
+
+// One slot of the device workspace: one head group's inputs, outputs and
+// backward workspace, each region 256-byte aligned.
+struct HostSlot {
+  size_t q, k, v, dO, o, lse, dq, dk, dv, ws, ws_bytes, total;
+};
+HostSlot host_slot(int hc, int N, int d) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t t = up(static_cast<size_t>(hc) * N * d * 2), l = up(static_cast<size_t>(hc) * N * 4);
+  HostSlot s;
+  size_t off = 0;
+  s.q = off, off += t;
+  s.k = off, off += t;
+  s.v = off, off += t;
+  s.dO = off, off += t;
+  s.o = off, off += t;
+  s.lse = off, off += l;
+  s.dq = off, off += t;
+  s.dk = off, off += t;
+  s.dv = off, off += t;
+  s.ws = off;
+  s.ws_bytes = up(fa_bwd_workspace_bytes(1, hc, N, d));
+  off += s.ws_bytes;
+  s.total = off;
+  return s;
+}
+
+int heads_per_group(int BH, int groups) {
+  const int g = groups < BH ? groups : BH;
+  return (BH + g - 1) / g;
+}
+}  // namespace
+
+extern "C" size_t fa_fwd_bwd_host_workspace_bytes(int B, int H, int N, int d, int groups) {
+  if (check_sizes(B, H, N, d) || groups < 1) return 0;
+  return kHostSlots * host_slot(heads_per_group(B * H, groups), N, d).total;
+}
+
+extern "C" int fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const void* dO, void* O, float* LSE,
+                               void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
+                               int groups, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, d);
+  if (rc) return rc;
+  if (groups < 1) return FA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !dO || !O || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
+  bool scale_ok = false;
+  (void)effective_scale(scale, d, &scale_ok);
+  if (!scale_ok) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_fwd_bwd_host_workspace_bytes(B, H, N, d, groups);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  const size_t tbytes = static_cast<size_t>(B) * H * N * d * 2, lbytes = static_cast<size_t>(B) * H * N * 4;
+  const Range ins[4] = {{(uintptr_t)Q, (uintptr_t)Q + tbytes},
+                        {(uintptr_t)K, (uintptr_t)K + tbytes},
+                        {(uintptr_t)V, (uintptr_t)V + tbytes},
+                        {(uintptr_t)dO, (uintptr_t)dO + tbytes}};
+  const Range outs[5] = {{(uintptr_t)O, (uintptr_t)O + tbytes},
+                         {(uintptr_t)LSE, (uintptr_t)LSE + lbytes},
+                         {(uintptr_t)dQ, (uintptr_t)dQ + tbytes},
+                         {(uintptr_t)dK, (uintptr_t)dK + tbytes},
+                         {(uintptr_t)dV, (uintptr_t)dV + tbytes}};
+  for (int a = 0; a < 5; ++a) {
+    for (int b = 0; b < 4; ++b)
+      if (overlaps(outs[a], ins[b])) return FA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 5; ++b)
+      if (overlaps(outs[a], outs[b])) return FA_ERR_INVALID_ARG;
+  }
+  int sms = 0;
+  if ((rc = device_ready(&sms))) return rc;
+  if (!is_device_ptr(workspace, need)) return FA_ERR_UNSUPPORTED_DEVICE;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& p = g_pipe[dev];
+  if (!host_pipe_ready(p)) {
+    g_last_cuda_error = static_cast<int>(cudaGetLastError());
+    return FA_ERR_LAUNCH;
+  }
+  clear_stale_error();
+  const int BH = B * H, hc = heads_per_group(BH, groups);
+  const int ng = (BH + hc - 1) / hc;
+  const HostSlot L = host_slot(hc, N, d);
+  const size_t head_t = static_cast<size_t>(N) * d * 2, head_l = static_cast<size_t>(N) * 4;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the pipeline starts after the work already queued on the caller's stream
+  cudaEventRecord(p.start, s);
+  cudaStreamWaitEvent(p.s_in, p.start, 0);
+  cudaStreamWaitEvent(p.s_run, p.start, 0);
+  cudaStreamWaitEvent(p.s_out, p.start, 0);
+  auto dptr = [&](int slot, size_t off) { return static_cast<uint8_t*>(workspace) + slot * L.total + off; };
+  for (int c = 0; c < ng; ++c) {
+    const int slot = c % kHostSlots;
+    const int h0 = c * hc, hn = (BH - h0) < hc ? (BH - h0) : hc;
+    const size_t nt = hn * head_t, nl = hn * head_l, ot = h0 * head_t, ol = h0 * head_l;
+    // copies in: the slot is free once group c - kHostSlots has been copied out
+    if (c >= kHostSlots) cudaStreamWaitEvent(p.s_in, p.ev_out[slot], 0);
+    const void* srcs[4] = {Q, K, V, dO};
+    const size_t dsts[4] = {L.q, L.k, L.v, L.dO};
+    for (int i = 0; i < 4; ++i)
+      cudaMemcpyAsync(dptr(slot, dsts[i]), static_cast<const uint8_t*>(srcs[i]) + ot, nt, cudaMemcpyDefault,
+                      p.s_in);
+    cudaEventRecord(p.ev_in[slot], p.s_in);
+    // forward and backward of the group's heads (B = 1, H = hn: the heads are contiguous)
+    cudaStreamWaitEvent(p.s_run, p.ev_in[slot], 0);
+    rc = fa_fwd(dptr(slot, L.q), dptr(slot, L.k), dptr(slot, L.v), dptr(slot, L.o),
+                reinterpret_cast<float*>(dptr(slot, L.lse)), 1, hn, N, d, causal, scale, p.s_run);
+    if (rc) return rc;
+    rc = fa_bwd(dptr(slot, L.q), dptr(slot, L.k), dptr(slot, L.v), dptr(slot, L.o), dptr(slot, L.dO),
+                reinterpret_cast<const float*>(dptr(slot, L.lse)), dptr(slot, L.dq), dptr(slot, L.dk),
+                dptr(slot, L.dv), 1, hn, N, d, causal, scale, dptr(slot, L.ws), L.ws_bytes, p.s_run);
+    if (rc) return rc;
+    cudaEventRecord(p.ev_run[slot], p.s_run);
+    // copies out
+    cudaStreamWaitEvent(p.s_out, p.ev_run[slot], 0);
+    cudaMemcpyAsync(static_cast<uint8_t*>(O) + ot, dptr(slot, L.o), nt, cudaMemcpyDefault, p.s_out);
+    cudaMemcpyAsync(reinterpret_cast<uint8_t*>(LSE) + ol, dptr(slot, L.lse), nl, cudaMemcpyDefault, p.s_out);
+    cudaMemcpyAsync(static_cast<uint8_t*>(dQ) + ot, dptr(slot, L.dq), nt, cudaMemcpyDefault, p.s_out);
+    cudaMemcpyAsync(static_cast<uint8_t*>(dK) + ot, dptr(slot, L.dk), nt, cudaMemcpyDefault, p.s_out);
+    cudaMemcpyAsync(static_cast<uint8_t*>(dV) + ot, dptr(slot, L.dv), nt, cudaMemcpyDefault, p.s_out);
+    cudaEventRecord(p.ev_out[slot], p.s_out);
+  }
+  // the caller's stream continues once the last copy out is done (which
+  // follows every copy in and kernel of the call)
+  cudaEventRecord(p.done, p.s_out);
+  cudaStreamWaitEvent(s, p.done, 0);
+  return launch_status();
+}

@@ -83,6 +83,10 @@ def load_library(build_if_missing: bool = True):
         lib.fa_fwd_kernel_name.restype = ctypes.c_char_p
         lib.fa_bwd_set_phase_events.argtypes = [vp, vp, vp, vp]
         lib.fa_bwd_set_phase_events.restype = None
+        lib.fa_fwd_bwd_host_workspace_bytes.argtypes = [i, i, i, i, i]
+        lib.fa_fwd_bwd_host_workspace_bytes.restype = sz
+        lib.fa_fwd_bwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+        lib.fa_fwd_bwd_host.restype = i
         lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
         lib.fa_selftest_wait_timeout.restype = i
         _lib = lib
@@ -265,6 +269,58 @@ def backward_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | N
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd_noalloc")
     return dq, dk, dv
+
+
+def host_workspace_bytes(B: int, H: int, N: int, d: int, groups: int) -> int:
+    return int(load_library().fa_fwd_bwd_host_workspace_bytes(B, H, N, d, groups))
+
+
+def _check_host(*ts):
+    t0 = ts[0]
+    if t0.dim() != 4:
+        raise ValueError("expected host tensors of shape [B, H, N, d]")
+    for t in ts:
+        if t.device.type != "cpu":
+            raise ValueError("host tensors must be CPU tensors")
+        if t.dtype != torch.bfloat16 or t.shape != t0.shape or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous bfloat16 of one shape")
+
+
+def forward_backward_host(q, k, v, do, causal: bool = False, scale: float | None = None, groups: int = 8,
+                          out=None, workspace=None, device=None):
+    """O, LSE, dQ, dK, dV of attention(q, k, v) with upstream gradient dO, from
+    host tensors [B, H, N, d] (bf16; page-locked for the copies to overlap) to
+    host tensors, through fa_fwd_bwd_host: head groups flow through copy-in,
+    kernels and copy-out at once.
+
+    `out`: optional preallocated host (o, lse, dq, dk, dv); `workspace`:
+    optional device buffer of host_workspace_bytes(B, H, N, d, groups) bytes.
+    The current stream of `device` waits for the whole pipeline, so the host
+    tensors hold the results once it synchronizes."""
+    _check_host(q, k, v, do)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    B, H, N, d = q.shape
+    if out is None:
+        pin = q.is_pinned()
+        mk = (lambda t: t.pin_memory()) if pin else (lambda t: t)
+        out = (mk(torch.empty_like(q)), mk(torch.empty((B, H, N), dtype=torch.float32)),
+               *(mk(torch.empty_like(q)) for _ in range(3)))
+    o, lse, dq, dk, dv = out
+    _check_host(o, dq, dk, dv)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or lse.device.type != "cpu" \
+            or not lse.is_contiguous():
+        raise ValueError("lse output must be a contiguous float32 CPU tensor [B, H, N]")
+    lib = load_library()
+    nbytes = int(lib.fa_fwd_bwd_host_workspace_bytes(B, H, N, d, groups))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    with _on(dev):
+        rc = lib.fa_fwd_bwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                                 int(bool(causal)), _scale(scale, d), int(groups), ws.data_ptr(), ws.numel(),
+                                 _stream_handle(dev))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_bwd_host")
+    return o, lse, dq, dk, dv
 
 
 def sync_status(device=None) -> int:

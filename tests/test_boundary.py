@@ -26,7 +26,7 @@ def test_every_declared_symbol_is_exported(lib):
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
                           "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name",
                           "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes", "fa_bwd_dkdv_kernel_name",
-                          "fa_bwd_deterministic"}
+                          "fa_bwd_deterministic", "fa_fwd_bwd_host", "fa_fwd_bwd_host_workspace_bytes"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:
@@ -183,3 +183,43 @@ def test_python_binding_refuses_cpu_tensors():
         fa.forward(q, q, q)
     with pytest.raises(ValueError):
         fa.forward(q.float(), q.float(), q.float())
+
+
+def test_host_pipeline_workspace_bytes(lib):
+    """Three slots, each one head group's Q, K, V, dO, O, dQ, dK, dV (bf16), LSE
+    (fp32) and backward workspace, every region rounded up to 256 bytes."""
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    def slot(hc, N, d):
+        t, l = up(hc * N * d * 2), up(hc * N * 4)
+        return 8 * t + l + up(lib.fa_bwd_workspace_bytes(1, hc, N, d))
+
+    assert lib.fa_fwd_bwd_host_workspace_bytes(2, 16, 4096, 128, 8) == 3 * slot(4, 4096, 128)
+    assert lib.fa_fwd_bwd_host_workspace_bytes(2, 3, 300, 64, 4) == 3 * slot(2, 300, 64)  # 6 heads -> groups of 2
+    assert lib.fa_fwd_bwd_host_workspace_bytes(1, 2, 100, 64, 50) == 3 * slot(1, 100, 64)  # clamped to B*H
+    assert lib.fa_fwd_bwd_host_workspace_bytes(1, 1, 100, 64, 0) == 0
+    assert lib.fa_fwd_bwd_host_workspace_bytes(1, 1, 0, 64, 1) == 0
+
+
+def _host(lib, ws=30 * A, ws_bytes=None, B=1, H=2, N=128, d=64, groups=2, **ptrs):
+    p = dict(q=A, k=2 * A, v=3 * A, do=4 * A, o=5 * A, lse=6 * A, dq=7 * A, dk=8 * A, dv=9 * A)
+    p.update(ptrs)
+    nb = lib.fa_fwd_bwd_host_workspace_bytes(B, H, N, d, groups) if ws_bytes is None else ws_bytes
+    return lib.fa_fwd_bwd_host(p["q"], p["k"], p["v"], p["do"], p["o"], p["lse"], p["dq"], p["dk"], p["dv"],
+                               B, H, N, d, 0, 0.0, groups, ws, nb, None)
+
+
+def test_host_pipeline_rejects_bad_arguments(lib):
+    assert _host(lib, N=0) == EINVAL
+    assert _host(lib, d=32) == EINVAL
+    assert _host(lib, groups=0) == EINVAL
+    assert _host(lib, q=0) == EINVAL
+    assert _host(lib, lse=0) == EINVAL
+    assert _host(lib, ws=0) == EWS
+    assert _host(lib, ws=30 * A + 8) == EWS
+    assert _host(lib, ws_bytes=1024) == EWS
+    assert _host(lib, o=A) == EINVAL              # O aliases Q
+    assert _host(lib, dv=8 * A) == EINVAL         # dV aliases dK
+    if not torch.cuda.is_available():
+        assert _host(lib) == EDEV                 # valid arguments: stops at the device check

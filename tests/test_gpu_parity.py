@@ -439,9 +439,10 @@ def test_forward_rescale_threshold(threshold, pair, monkeypatch):
 
 
 def test_host_pipeline_equals_the_device_path():
-    """forward_backward_host (pinned host tensors, heads in groups through
-    three streams) returns exactly the device path's outputs: the same
-    kernels on the same heads, only the copies are scheduled differently."""
+    """fa_fwd_bwd_host (host tensors in and out, head groups through copy-in,
+    kernels and copy-out on the library's streams) returns the device path's
+    outputs: the same kernels on the same heads; only dQ's partial sums may
+    be added in another order.  Page-locked and ordinary host memory alike."""
     from io_aware_tiled_b200.host_pipeline import forward_backward_host
     dev = _dev()
     B, H, N, d = 2, 3, 300, 128
@@ -449,13 +450,16 @@ def test_host_pipeline_equals_the_device_path():
     for causal in (False, True):
         o, lse = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal)
         g = fa.backward(q.to(dev), k.to(dev), v.to(dev), o, do.to(dev), lse, causal)
-        host = forward_backward_host(*(t.pin_memory() for t in (q, k, v, do)), causal, groups=4, device=dev)
-        torch.cuda.synchronize()
-        assert fa.sync_status() == fa.FA_OK
-        for i, (got, want) in enumerate(zip(host, (o, lse, *g))):
-            if i == 2:  # dQ: partial sums added in a varying order
-                assert_same_up_to_summation_order(got, want, f"host pipeline dQ causal={causal}")
-            else:
-                assert torch.equal(got, want.cpu())
+        for pinned, groups in ((True, 4), (False, 1), (True, 6), (True, 100)):
+            ins = [t.pin_memory() if pinned else t for t in (q, k, v, do)]
+            host = forward_backward_host(*ins, causal, groups=groups, device=dev)
+            torch.cuda.synchronize()
+            assert fa.sync_status() == fa.FA_OK
+            for i, (got, want) in enumerate(zip(host, (o, lse, *g))):
+                what = f"host pipeline causal={causal} pinned={pinned} groups={groups} output {i}"
+                if i == 2:  # dQ: partial sums added in a varying order
+                    assert_same_up_to_summation_order(got, want, what)
+                else:
+                    assert torch.equal(got, want.cpu()), what
     with pytest.raises(ValueError):
-        forward_backward_host(q, k, v, do)  # not pinned
+        forward_backward_host(q.to(dev), k, v, do)  # a device tensor where host memory is expected
