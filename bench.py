@@ -304,6 +304,10 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # sha256 of the sources the kernel is compiled from at capture time: once they
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
+    # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal_dram.md (32 heads)
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.785408e6 + 14.962176e6) / 32,
+                          "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
+                          "sha256": "0397850b9e760068165f4e5a374267e6c5ac9330881a9a4d139d2c46c6c72456"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
     "fa_bwd_fused_kernel": {"bytes_per_head": (202.540544e6 + 86.772480e6) / 32,

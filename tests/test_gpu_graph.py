@@ -1,6 +1,8 @@
 """The library's calls can be captured in a CUDA graph and replayed: they are
 asynchronous on the caller's stream, allocate nothing (given a workspace), and
-bake their tensor maps into the launches' parameters."""
+bake their tensor maps into the launches' parameters.  Replays reproduce the
+eager outputs exactly, except dQ of the default backward, whose partial sums
+are added in an order that can vary from run to run."""
 from __future__ import annotations
 
 import pytest
@@ -8,6 +10,7 @@ import torch
 
 from io_aware_tiled_b200 import fa
 from io_aware_tiled_b200.inputs import attention_inputs
+from tests.parity import assert_same_up_to_summation_order
 
 pytestmark = pytest.mark.gpu
 
@@ -44,5 +47,8 @@ def test_graph_replay_matches_eager():
         g.replay()
         torch.cuda.synchronize()
         assert fa.sync_status() == fa.FA_OK
-        for got, ref in zip((o, lse, dq, dk, dv), want):
-            assert torch.equal(got, ref)
+        for i, (got, ref) in enumerate(zip((o, lse, dq, dk, dv), want)):
+            if i == 2:  # dQ: the backward adds its partial sums in a varying order
+                assert_same_up_to_summation_order(got, ref, "graph replay dQ")
+            else:
+                assert torch.equal(got, ref)
