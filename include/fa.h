@@ -59,7 +59,9 @@ typedef enum {
  * In:  Q, K, V [B,H,N,d] bf16.
  * Out: O [B,H,N,d] bf16 (O = P V, rounded to nearest even), LSE [B,H,N] fp32.
  * One persistent kernel launch on `stream`: CTA pairs (fa_fwd_2sm_kernel) for
- * d = 128 without the mask, one SM per CTA (fa_fwd_kernel) otherwise.  Two
+ * d = 128 without the mask, one SM per CTA (fa_fwd_kernel) otherwise.  With
+ * the mask the launch carries each CTA's list of query-tile pairs, computed on
+ * the host at the first call for a shape and kept (a few shapes at a time).  Two
  * environment variables, read at each call, select other forms for
  * comparisons: FA_FWD_PAIR=0 / =1 forces the one-SM / paired kernel for
  * d = 128; FA_FWD_BN=64 runs the one-SM kernel with 64-key K/V tiles instead

@@ -1,7 +1,11 @@
 // fa_api.cu -- the C ABI of libfa.so: argument validation, TMA descriptor
 // encoding and kernel launches for the sm_100a attention kernels.
 #include <math.h>
+#include <algorithm>
 #include <mutex>
+#include <queue>
+#include <utility>
+#include <vector>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -286,6 +290,74 @@ float effective_scale(float scale, int d, bool* ok) {
   return scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(d));
 }
 
+// Unit lists of the causal one-SM forward.  A unit is a pair of 128-row query
+// tiles of one head; pair p of a head runs (2p+1) + (2p+2) key-tile steps
+// (scaled by 128 / BN), plus about one step per query tile of fixed cost.
+// Order: heads in groups whose K and V fit in 64 MiB of L2, inside a group the
+// longest units first; then a longest-processing-time assignment: each unit
+// in that order goes to the CTA with the least work so far.  Each CTA runs its
+// units in assignment order.  Lists are cached per shape (they depend only on
+// the head count, N, d, the key tile and the grid).
+struct UnitListEntry {
+  int BH = -1, N = 0, d = 0, bn = 0, grid = 0;
+  fa::FwdUnitList list;
+};
+constexpr int kListCache = 4;
+UnitListEntry g_lists[kListCache];
+int g_lists_next = 0;
+std::mutex g_lists_mu;
+
+constexpr long long kFwdGroupBytes = 64ll << 20;  // K and V of a head group
+
+bool build_unit_list(fa::FwdUnitList* L, int BH, int N, int d, int bn, int grid) {
+  const int NKT = (N + bn - 1) / bn, NQT = (N + 127) / 128, NP = (NQT + 1) / 2, R = 128 / bn;
+  const long long units = static_cast<long long>(BH) * NP;
+  if (units > fa::FwdUnitList::kMaxUnits || grid > fa::FwdUnitList::kMaxCtas || grid < 1) return false;
+  const long long per_head = 4ll * N * d;  // K and V, bf16
+  long long g = kFwdGroupBytes / per_head;
+  const int G = g >= BH ? BH : (g < 1 ? 1 : static_cast<int>(g));
+  std::vector<int> order;
+  order.reserve(units);
+  for (int g0 = 0; g0 < BH; g0 += G)
+    for (int r = 0; r < NP; ++r)
+      for (int bh = g0; bh < BH && bh < g0 + G; ++bh) order.push_back(r * BH + bh);
+  using Load = std::pair<long long, int>;  // (work so far, CTA): the smallest on top
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < grid; ++c) heap.push({0, c});
+  std::vector<int> owner(order.size()), count(grid, 0);
+  for (size_t i = 0; i < order.size(); ++i) {
+    const int qp = NP - 1 - order[i] / BH;
+    const int nk0 = std::min((2 * qp + 1) * R, NKT), nk1 = std::min((2 * qp + 2) * R, NKT);
+    Load top = heap.top();
+    heap.pop();
+    owner[i] = top.second;
+    ++count[top.second];
+    heap.push({top.first + nk0 + nk1 + 2 * R, top.second});
+  }
+  L->n = static_cast<int>(order.size());
+  L->start[0] = 0;
+  for (int c = 0; c < grid; ++c) L->start[c + 1] = static_cast<unsigned short>(L->start[c] + count[c]);
+  std::vector<int> fill(L->start, L->start + grid);
+  for (size_t i = 0; i < order.size(); ++i) L->order[fill[owner[i]]++] = static_cast<unsigned short>(order[i]);
+  return true;
+}
+
+// The list for a causal launch, copied into *out; false: use the serpentine deal.
+bool causal_unit_list(fa::FwdUnitList* out, int BH, int N, int d, int bn, int grid) {
+  std::lock_guard<std::mutex> lock(g_lists_mu);
+  for (const UnitListEntry& e : g_lists)
+    if (e.BH == BH && e.N == N && e.d == d && e.bn == bn && e.grid == grid) {
+      *out = e.list;
+      return e.list.n > 0;
+    }
+  UnitListEntry& e = g_lists[g_lists_next];
+  g_lists_next = (g_lists_next + 1) % kListCache;
+  e.BH = BH, e.N = N, e.d = d, e.bn = bn, e.grid = grid;
+  if (!build_unit_list(&e.list, BH, N, d, bn, grid)) e.list.n = 0;
+  *out = e.list;
+  return e.list.n > 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -388,24 +460,27 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   const float sl2 = sc * fa::kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* o = static_cast<__nv_bfloat16*>(O);
+  fa::FwdUnitList ul;  // causal: this shape's unit lists (n = 0: serpentine deal)
+  ul.n = 0;
+  if (causal) causal_unit_list(&ul, BH, N, d, fwd_key_tile(), grid);
   if (fwd_key_tile() == 64) {  // 64-key tiles: for tile-size comparisons only
     CUtensorMap mk64, mv64;
     if (!make_map(&mk64, K, BH, N, d, 64) || !make_map(&mv64, V, BH, N, d, 64)) return encode_failed();
     if (d == 64) {
-      if (causal) fa::fa_fwd_kernel<64, true, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
-      else fa::fa_fwd_kernel<64, false, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
+      if (causal) fa::fa_fwd_kernel<64, true, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale, ul);
+      else fa::fa_fwd_kernel<64, false, 64><<<grid, fa::FwdCfg<64, 64>::THREADS, fa::FwdCfg<64, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale, fa::FwdNoList{0});
     } else {
-      if (causal) fa::fa_fwd_kernel<128, true, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
-      else fa::fa_fwd_kernel<128, false, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale);
+      if (causal) fa::fa_fwd_kernel<128, true, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale, ul);
+      else fa::fa_fwd_kernel<128, false, 64><<<grid, fa::FwdCfg<128, 64>::THREADS, fa::FwdCfg<128, 64>::SMEM_BYTES, s>>>(mq, mk64, mv64, o, LSE, BH, N, sl2, rescale, fa::FwdNoList{0});
     }
     return launch_status();
   }
   if (d == 64) {
-    if (causal) fa::fa_fwd_kernel<64, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
-    else fa::fa_fwd_kernel<64, false><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
+    if (causal) fa::fa_fwd_kernel<64, true><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale, ul);
+    else fa::fa_fwd_kernel<64, false><<<grid, fa::FwdCfg<64>::THREADS, fa::FwdCfg<64>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale, fa::FwdNoList{0});
   } else {
-    if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
-    else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale);
+    if (causal) fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale, ul);
+    else fa::fa_fwd_kernel<128, false><<<grid, fa::FwdCfg<128>::THREADS, fa::FwdCfg<128>::SMEM_BYTES, s>>>(mq, mk, mv, o, LSE, BH, N, sl2, rescale, fa::FwdNoList{0});
   }
   return launch_status();
 }

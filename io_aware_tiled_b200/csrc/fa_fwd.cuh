@@ -84,10 +84,15 @@ enum FwdWaitSite : unsigned int {
 };
 
 // Unit order.  Non-causal: head-major, so the CTAs running at the same time
-// share a few heads' K and V in L2.  Causal: longest units (last query pairs)
-// first across all heads, dealt in serpentine order (serpentine_unit), so the
-// persistent CTAs finish together.  (Grouping heads to keep K and V in L2, as
-// the backward does, breaks the global longest-first sort and costs more.)
+// share a few heads' K and V in L2, dealt in serpentine order.  Causal: unit u
+// is rank u / BH (0 = the longest, the last query pair) of head u % BH; the
+// host gives each CTA its list of units (FwdUnitList): heads in groups whose K
+// and V fit in L2, longest units first inside a group, each unit assigned to
+// the CTA with the least work so far.  A static deal of that grouped order
+// would leave some CTAs with far more work; the assignment keeps both the
+// balance of a global longest-first deal and the L2 locality of the groups.
+// Without a list (more units or CTAs than it holds) the causal units are
+// dealt longest first, in serpentine order.
 __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool causal, int& bh, int& qp) {
   if (causal) {
     const int r = u / BH;
@@ -99,12 +104,46 @@ __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool caus
   }
 }
 
+// Per-CTA unit lists of the causal forward, computed on the host (a
+// longest-processing-time assignment over an L2-friendly unit order) and
+// passed by value.  n = 0: no list; the units are dealt in serpentine order.
+struct FwdUnitList {
+  static constexpr int kMaxCtas = 160;
+  static constexpr int kMaxUnits = 4096;
+  int n;                                   // units in `order`
+  unsigned short start[kMaxCtas + 1];      // CTA c takes order[start[c] .. start[c + 1])
+  unsigned short order[kMaxUnits];         // unit indices as fwd_decode_unit reads them
+};
+struct FwdNoList {
+  int n;
+};
+template <bool CAUSAL>
+struct FwdListOf {
+  using type = FwdNoList;
+};
+template <>
+struct FwdListOf<true> {
+  using type = FwdUnitList;
+};
+
+// The k-th unit of this CTA (>= units when it has no more).
+template <typename L>
+__device__ __forceinline__ int fwd_unit(const L& list, int k, int units) {
+  if constexpr (sizeof(L) > sizeof(FwdNoList)) {
+    if (list.n > 0) {
+      const int i = list.start[blockIdx.x] + k;
+      return i < list.start[blockIdx.x + 1] ? static_cast<int>(list.order[i]) : units;
+    }
+  }
+  return serpentine_unit(k, blockIdx.x, gridDim.x);
+}
+
 template <int D, bool CAUSAL, int BN_ = 128>
 __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
                   float* __restrict__ LSE, int BH, int N, float scale_log2,
-                  float rescale_log2) {
+                  float rescale_log2, const __grid_constant__ typename FwdListOf<CAUSAL>::type list) {
   using C = FwdCfg<D, BN_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -160,7 +199,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t kv_it = 0, q_it = 0;
-      for (int k = 0, u = blockIdx.x; u < units; u = serpentine_unit(++k, blockIdx.x, gridDim.x)) {
+      for (int k = 0, u = fwd_unit(list, 0, units); u < units; u = fwd_unit(list, ++k, units)) {
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
         const int nk1 = CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT;
@@ -217,7 +256,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
       };
       uint32_t kv_it = 0, q_it = 0, unit_it = 0;
       uint32_t p_ph0 = 0, p_ph1 = 0;
-      for (int k = 0, u = blockIdx.x; u < units; u = serpentine_unit(++k, blockIdx.x, gridDim.x), ++unit_it) {
+      for (int k = 0, u = fwd_unit(list, 0, units); u < units; u = fwd_unit(list, ++k, units), ++unit_it) {
         int bh, qp;
         fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
         (void)bh;
@@ -307,7 +346,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
     const uint32_t bar_o = bars + 8 * (C::B_O_FULL + wg), bar_oe = bars + 8 * (C::B_O_EMPTY + wg);
     uint32_t s_it = 0, o_it = 0;
     bool ok = true;
-    for (int k = 0, u = blockIdx.x; u < units && ok; u = serpentine_unit(++k, blockIdx.x, gridDim.x)) {
+    for (int k = 0, u = fwd_unit(list, 0, units); u < units && ok; u = fwd_unit(list, ++k, units)) {
       int bh, qp;
       fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
       const int qt = 2 * qp + wg;
