@@ -66,6 +66,24 @@ def test_forward_matches_oracle(B, H, N, d, causal, sigma):
     check_lse(f64(lse), rl, f"fwd {B,H,N,d,causal}")
 
 
+def test_causal_forward_beyond_the_unit_lists():
+    """Causal launches normally follow per-CTA unit lists computed on the host;
+    with more than 4096 query-tile pairs (here 1200 heads x 8) the units are
+    dealt in serpentine order instead.  Sampled rows of every region against
+    the oracle, the first row of every head exactly V[0]."""
+    dev = _dev()
+    B, H, N, d = 4, 300, 2048, 64
+    q, k, v, _ = attention_inputs(B, H, N, d, seed=17, with_do=False)
+    o, lse = _run_fwd(q, k, v, True)
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([rng.choice(B * H * N, 300, replace=False),
+                                     np.arange(0, B * H * N, N) + N - 1]))
+    ro, rl = oracle.forward_rows(f64(q), f64(k), f64(v), True, 1 / d ** 0.5, rows)
+    check_o(f64(o).reshape(-1, d)[rows], ro, "causal, 9600 units")
+    check_lse(f64(lse).reshape(-1)[rows], rl, "causal, 9600 units")
+    assert torch.equal(o[:, :, 0].cpu(), v[:, :, 0])
+
+
 def test_forward_explicit_scale_and_default():
     q, k, v, _ = attention_inputs(1, 2, 200, 128, seed=5, with_do=False)
     for scale in (0.05, 0.3):
