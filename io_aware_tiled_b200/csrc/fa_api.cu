@@ -965,11 +965,11 @@ extern "C" int fa_fwd_bwd_host(const void* Q, const void* K, const void* V, cons
     cudaStreamWaitEvent(p.s_run, p.ev_in[slot], 0);
     rc = fa_fwd(dptr(slot, L.q), dptr(slot, L.k), dptr(slot, L.v), dptr(slot, L.o),
                 reinterpret_cast<float*>(dptr(slot, L.lse)), 1, hn, N, d, causal, scale, p.s_run);
-    if (rc) return rc;
-    rc = fa_bwd(dptr(slot, L.q), dptr(slot, L.k), dptr(slot, L.v), dptr(slot, L.o), dptr(slot, L.dO),
-                reinterpret_cast<const float*>(dptr(slot, L.lse)), dptr(slot, L.dq), dptr(slot, L.dk),
-                dptr(slot, L.dv), 1, hn, N, d, causal, scale, dptr(slot, L.ws), L.ws_bytes, p.s_run);
-    if (rc) return rc;
+    if (!rc)
+      rc = fa_bwd(dptr(slot, L.q), dptr(slot, L.k), dptr(slot, L.v), dptr(slot, L.o), dptr(slot, L.dO),
+                  reinterpret_cast<const float*>(dptr(slot, L.lse)), dptr(slot, L.dq), dptr(slot, L.dk),
+                  dptr(slot, L.dv), 1, hn, N, d, causal, scale, dptr(slot, L.ws), L.ws_bytes, p.s_run);
+    if (rc) break;  // no copy out of this group; the work already queued is still joined below
     cudaEventRecord(p.ev_run[slot], p.s_run);
     // copies out
     cudaStreamWaitEvent(p.s_out, p.ev_run[slot], 0);
@@ -980,9 +980,15 @@ extern "C" int fa_fwd_bwd_host(const void* Q, const void* K, const void* V, cons
     cudaMemcpyAsync(static_cast<uint8_t*>(dV) + ot, dptr(slot, L.dv), nt, cudaMemcpyDefault, p.s_out);
     cudaEventRecord(p.ev_out[slot], p.s_out);
   }
-  // the caller's stream continues once the last copy out is done (which
-  // follows every copy in and kernel of the call)
+  // the caller's stream continues once everything this call queued is done
+  // (on error too, so that no copy into the caller's buffers outlives the
+  // stream order the caller sees)
+  cudaEventRecord(p.done, p.s_in);
+  cudaStreamWaitEvent(p.s_out, p.done, 0);
+  cudaEventRecord(p.done, p.s_run);
+  cudaStreamWaitEvent(p.s_out, p.done, 0);
   cudaEventRecord(p.done, p.s_out);
   cudaStreamWaitEvent(s, p.done, 0);
-  return launch_status();
+  const int st = launch_status();
+  return rc ? rc : st;
 }
