@@ -479,5 +479,20 @@ def test_host_pipeline_equals_the_device_path():
                     assert_same_up_to_summation_order(got, want, what)
                 else:
                     assert torch.equal(got, want.cpu()), what
+    # 16 heads in four groups of 4: more groups than the pipeline's three slots
+    B, H, N, d = 2, 8, 200, 64
+    q, k, v, do = attention_inputs(B, H, N, d, seed=78)
+    for causal in (False, True):
+        o, lse = fa.forward(q.to(dev), k.to(dev), v.to(dev), causal)
+        g = fa.backward(q.to(dev), k.to(dev), v.to(dev), o, do.to(dev), lse, causal)
+        host = forward_backward_host(*(t.pin_memory() for t in (q, k, v, do)), causal, groups=4, device=dev)
+        torch.cuda.synchronize()
+        assert fa.sync_status() == fa.FA_OK
+        for i, (got, want) in enumerate(zip(host, (o, lse, *g))):
+            what = f"host pipeline 16 heads causal={causal} output {i}"
+            if i == 2:
+                assert_same_up_to_summation_order(got, want, what)
+            else:
+                assert torch.equal(got, want.cpu()), what
     with pytest.raises(ValueError):
         forward_backward_host(q.to(dev), k, v, do)  # a device tensor where host memory is expected
