@@ -27,7 +27,13 @@
 //     and O_t += P_t V_j (M=128, N=d, K=128) with P_t read from TENSOR MEMORY
 //     (bf16, written over S_t's columns) and V_j MN-major from shared memory.
 //   * Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1
-//     [128,256), O0 [256, 256+d), O1 [256+d, 256+2d).
+//     [128,256), O0 [256, 256+d), O1 [256+d, 256+2d).  At d = 128 S_t is Q
+//     tile t's buffer: a tile's next S waits until its PV has read P.  At
+//     d = 64 the free columns [384,512) hold a third buffer S2 and the three
+//     form a ring over the unit's tiles in issue order, so a Q tile's next S
+//     is computed while its softmax still runs; before rescaling O the
+//     softmax then waits for its previous PV (an O_DONE barrier per Q tile
+//     and PV-count parity).
 //   * Softmax: each thread owns one full row of S (tcgen05.ld 32x32b), so the
 //     row max and row sum are register reductions.  Work is in base 2 with
 //     scale*log2(e) folded into one FMA.  O is rescaled only when a row's max
@@ -61,12 +67,18 @@ struct FwdCfg {
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = NQB;
   static constexpr int B_K_FULL = 2 * NQB, B_K_EMPTY = 2 * NQB + ST, B_V_FULL = 2 * NQB + 2 * ST,
                        B_V_EMPTY = 2 * NQB + 3 * ST;
-  static constexpr int B_S_FULL = 2 * NQB + 4 * ST, B_P_FULL = B_S_FULL + 2, B_O_FULL = B_P_FULL + 2,
-                       B_O_EMPTY = B_O_FULL + 2;
-  static constexpr int NUM_BARS = B_O_EMPTY + 2;
+  // S buffers: two (one per Q tile) at d = 128; at d = 64 with 128-key tiles
+  // a ring of three over the unit's tiles in issue order (the spare tensor
+  // memory after O0 and O1 holds the third)
+  static constexpr int NS = (D == 64 && BN == 128) ? 3 : 2;
+  static constexpr int B_S_FULL = 2 * NQB + 4 * ST, B_P_FULL = B_S_FULL + NS, B_O_FULL = B_P_FULL + NS,
+                       B_O_EMPTY = B_O_FULL + 2, B_O_DONE = B_O_EMPTY + 2;  // O_DONE: [Q tile][PV count & 1]
+  static constexpr int NUM_BARS = B_O_DONE + 4;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;  // + room to align the base to 1024
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = BN, TM_O0 = 256, TM_O1 = 256 + D;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = BN, TM_O0 = 256, TM_O1 = 256 + D, TM_S2 = 384;
+  static_assert(NS == 2 || TM_O1 + D <= TM_S2, "third S buffer overlaps O");
+  __host__ __device__ static constexpr uint32_t tm_s(int b) { return b == 0 ? TM_S0 : (b == 1 ? TM_S1 : TM_S2); }
   static constexpr uint32_t TMEM_COLS = 512;
   // warpgroup 0: warp 0 TMA, warp 1 MMA, warps 2-3 idle; warpgroups 1 and 2: softmax of Q tile 0 and 1
   static constexpr int THREADS = 384;
@@ -101,6 +113,21 @@ __device__ __forceinline__ void fwd_decode_unit(int u, int BH, int NP, bool caus
   } else {
     bh = u / NP;
     qp = u - bh * NP;
+  }
+}
+
+// Order of a unit's tiles in the S-buffer ring (three buffers, d = 64): key
+// tile j of Q tile 0, then key tile j of Q tile 1, for j < nk0; then Q tile 1
+// alone for its last nk1 - nk0 key tiles (causal).  Tile i of a CTA's whole
+// sequence uses buffer i % 3.
+__device__ __forceinline__ int ring_pos(int j, int t, int nk0) { return j < nk0 ? 2 * j + t : nk0 + j; }
+__device__ __forceinline__ void ring_tile(int i, int nk0, int& j, int& t) {
+  if (i < 2 * nk0) {
+    j = i >> 1;
+    t = i & 1;
+  } else {
+    j = i - nk0;
+    t = 1;
   }
 }
 
@@ -164,11 +191,15 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
       mbar_init(bars + 8 * (C::B_V_FULL + s), 1);
       mbar_init(bars + 8 * (C::B_V_EMPTY + s), 1);
     }
+    for (int b = 0; b < C::NS; ++b) {
+      mbar_init(bars + 8 * (C::B_S_FULL + b), 1);
+      mbar_init(bars + 8 * (C::B_P_FULL + b), 128);
+    }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bars + 8 * (C::B_S_FULL + t), 1);
-      mbar_init(bars + 8 * (C::B_P_FULL + t), 128);
       mbar_init(bars + 8 * (C::B_O_FULL + t), 1);
       mbar_init(bars + 8 * (C::B_O_EMPTY + t), 128);
+      mbar_init(bars + 8 * (C::B_O_DONE + 2 * t), 1);
+      mbar_init(bars + 8 * (C::B_O_DONE + 2 * t + 1), 1);
     }
     fence_mbar_init();
   }
@@ -255,6 +286,67 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           mma_ts_k64(d_tmem, p_tmem, vd, IDESC_PV, acc ? 1u : 0u);
       };
       uint32_t kv_it = 0, q_it = 0, unit_it = 0;
+      if constexpr (C::NS == 3) {
+        // Ring of three S buffers: after PV of tile i the MMA of tile i + 3
+        // goes into the buffer P_i occupied, so each Q tile's next S is ready
+        // while its softmax still runs.
+        uint32_t g0 = 0, pv0 = 0, pv1 = 0;  // ring tiles before this unit; PVs issued per Q tile
+        for (int k = 0, u = fwd_unit(list, 0, units); u < units; u = fwd_unit(list, ++k, units), ++unit_it) {
+          int bh, qp;
+          fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
+          (void)bh;
+          const int nk0 = CAUSAL ? min((2 * qp + 1) * C::R, NKT) : NKT;
+          const int nk1 = CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT;
+          const int n = nk0 + nk1;
+          const int qb = q_it % C::NQB;
+          const uint32_t sQb = sQ + qb * 2 * C::Q_TILE;
+          bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_FULL + qb), (q_it / C::NQB) & 1, FW_MMA_Q));
+          ++q_it;
+          if (!ok) break;
+          tc_fence_after();
+          // S of the unit's ring tile i into its buffer; K_j is free after Q tile 1's S
+          auto s_of = [&](int i) -> bool {
+            int j, t;
+            ring_tile(i, nk0, j, t);
+            const uint32_t it = kv_it + j;
+            const int s = it % C::ST;
+            if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_K_FULL + s), (it / C::ST) & 1, FW_MMA_K)))
+              return false;
+            tc_fence_after();
+            const int b = (g0 + i) % C::NS;
+            issue_s(tmem + C::tm_s(b), sQb + t * C::Q_TILE, sK + s * C::KV_TILE);
+            tc_commit_warp(bars + 8 * (C::B_S_FULL + b));
+            if (t == 1) tc_commit_warp(bars + 8 * (C::B_K_EMPTY + s));
+            return true;
+          };
+          for (int i = 0; i < n && i < C::NS && ok; ++i) ok = s_of(i);
+          for (int i = 0; i < n && ok; ++i) {
+            int j, t;
+            ring_tile(i, nk0, j, t);
+            const uint32_t it = kv_it + j, g = g0 + i;
+            const int s = it % C::ST, b = g % C::NS;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_V_FULL + s), (it / C::ST) & 1, FW_MMA_V))))
+              break;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + b), (g / C::NS) & 1, FW_MMA_P))))
+              break;
+            if (j == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_O_EMPTY + t), (unit_it & 1) ^ 1,
+                                                                     FW_MMA_OE))))
+              break;
+            tc_fence_after();
+            issue_pv(tmem + (t ? C::TM_O1 : C::TM_O0), tmem + C::tm_s(b), sV + s * C::KV_TILE, j > 0);
+            const uint32_t pc = t ? pv1 : pv0;
+            tc_commit_warp(bars + 8 * (C::B_O_DONE + 2 * t + (pc & 1)));
+            if (t) ++pv1; else ++pv0;
+            if (t == 1) tc_commit_warp(bars + 8 * (C::B_V_EMPTY + s));
+            if (j == (t ? nk1 : nk0) - 1) tc_commit_warp(bars + 8 * (C::B_O_FULL + t));
+            if (i + C::NS < n) ok = s_of(i + C::NS);
+          }
+          if (!ok) break;
+          tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));
+          kv_it += nk1;
+          g0 += n;
+        }
+      } else {
       uint32_t p_ph0 = 0, p_ph1 = 0;
       for (int k = 0, u = fwd_unit(list, 0, units); u < units; u = fwd_unit(list, ++k, units), ++unit_it) {
         int bh, qp;
@@ -319,6 +411,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
         tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));
         kv_it += nk1;
       }
+      }
       // The last unit's Q_EMPTY arrival is the last one this thread's commits
       // make; wait for it so no arrival lands after the CTA has exited.
       if (q_it > 0)
@@ -345,22 +438,34 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
     const uint32_t bar_s = bars + 8 * (C::B_S_FULL + wg), bar_p = bars + 8 * (C::B_P_FULL + wg);
     const uint32_t bar_o = bars + 8 * (C::B_O_FULL + wg), bar_oe = bars + 8 * (C::B_O_EMPTY + wg);
     uint32_t s_it = 0, o_it = 0;
+    uint32_t g0 = 0, pv_c = 0;  // three-buffer ring: ring tiles before this unit; this Q tile's tiles so far
     bool ok = true;
     for (int k = 0, u = fwd_unit(list, 0, units); u < units && ok; u = fwd_unit(list, ++k, units)) {
       int bh, qp;
       fwd_decode_unit(u, BH, NP, CAUSAL, bh, qp);
       const int qt = 2 * qp + wg;
       const int nk = CAUSAL ? min((qt + 1) * C::R, NKT) : NKT;
+      const int nk0 = CAUSAL ? min((2 * qp + 1) * C::R, NKT) : NKT;  // Q tile 0's key tiles
       const int row = qt * C::BM + r;
       float m_ref = -INFINITY, l = 0.f;
-      for (int j = 0; j < nk; ++j) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s, s_it & 1, FW_SM_S)))) break;
+      for (int j = 0; j < nk; ++j, ++pv_c) {
+        // this tile's S buffer and barriers
+        uint32_t tS_j = tS, bar_s_j = bar_s, bar_p_j = bar_p, s_ph = s_it & 1;
+        if constexpr (C::NS == 3) {
+          const uint32_t g = g0 + ring_pos(j, wg, nk0);
+          const int b = g % C::NS;
+          tS_j = tmem + lane_off + C::tm_s(b);
+          bar_s_j = bars + 8 * (C::B_S_FULL + b);
+          bar_p_j = bars + 8 * (C::B_P_FULL + b);
+          s_ph = (g / C::NS) & 1;
+        }
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s_j, s_ph, FW_SM_S)))) break;
         ++s_it;
         tc_fence_after();
         constexpr int NC = C::BN;  // score columns per row
         uint32_t sr[NC];
 #pragma unroll
-        for (int c = 0; c < NC / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        for (int c = 0; c < NC / 32; ++c) tmem_ld32(tS_j + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < NC / 32; ++c) reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
@@ -402,16 +507,24 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
             ps[c & 7] += p0 + p1;
             p[c] = pack_bf16(p0, p1);
           }
-          tmem_st16(tS + ch * 16, p);
+          tmem_st16(tS_j + ch * 16, p);
         }
 #pragma unroll
         for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
           for (int e = 0; e < w; ++e) ps[e] += ps[e + w];
         const float lsum = ps[0];
-        // O holds PV of tiles 0..j-1 (the S MMA that signalled s_full was issued
-        // after them); rescale it before this tile's PV is issued.
+        // Rescale O before this tile's PV is issued.  With two S buffers O holds
+        // PV of tiles 0..j-1 already (the S MMA that signalled s_full was issued
+        // after them); with the ring, wait for the PV of tile j-1 first.
         if (warp_rescale && j > 0) {
+          if constexpr (C::NS == 3) {
+            const uint32_t pc = pv_c - 1;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_O_DONE + 2 * wg + (pc & 1)),
+                                                         (pc >> 1) & 1, FW_SM_O))))
+              break;
+            tc_fence_after();
+          }
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -425,10 +538,11 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar_p);
+        mbar_arrive(bar_p_j);
         l += lsum;
       }
       if (!ok) break;
+      g0 += nk0 + (CAUSAL ? min((2 * qp + 2) * C::R, NKT) : NKT);
       // epilogue: O / l (bf16) and LSE (fp32, natural log of the scaled logits)
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_o, o_it & 1, FW_SM_O)))) break;
       ++o_it;
