@@ -86,8 +86,9 @@ struct FwdCfg {
   // softmax warpgroups 208 each (128 x 64 + 256 x 208 = 61440)
   static constexpr uint32_t REGS_CONTROL = 64, REGS_SOFTMAX = 208;
   // one exponential pair in EXP_EMUL_EVERY goes to exp2_poly3 (FMA pipe)
-  // instead of the MUFU: 1/4 of them at d = 64, 1/8 at d = 128 (measured best)
-  static constexpr int EXP_EMUL_EVERY = (D == 64) ? 4 : 8;
+  // instead of the MUFU: 1/16 of them at d = 64 (with the S ring the
+  // softmax's issue slots, not the MUFU, bound it), 1/8 at d = 128 (measured best)
+  static constexpr int EXP_EMUL_EVERY = (D == 64) ? 16 : 8;
 };
 
 // wait-site identifiers recorded in the error word
