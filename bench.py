@@ -310,9 +310,9 @@ NCU_TRAFFIC = {
                           "sha256": "0397850b9e760068165f4e5a374267e6c5ac9330881a9a4d139d2c46c6c72456"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
-    "fa_bwd_fused_kernel": {"bytes_per_head": (202.540544e6 + 86.772480e6) / 32,
+    "fa_bwd_fused_kernel": {"bytes_per_head": (202.848256e6 + 85.483776e6) / 32,
                             "sources": ("fa_bwd_fused.cuh", "fa_device.cuh"),
-                            "sha256": "8dab14cec0ee2fc62a21f534d140f5bc794e235b6ef798c6fa0e0184840fd84d"},
+                            "sha256": "6dcc818fafe19c681afbcb02cf6c9b2353c6bbdc8702fbd8717d313396218810"},
 }
 
 

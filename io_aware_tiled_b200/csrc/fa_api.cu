@@ -309,6 +309,28 @@ std::mutex g_lists_mu;
 
 constexpr long long kFwdGroupBytes = 64ll << 20;  // K and V of a head group
 
+// Longest-processing-time assignment of units, taken in the given order (the
+// caller puts the longest first), each to the CTA with the least work so far;
+// each CTA runs its units in assignment order.
+void lpt_assign(fa::UnitList* L, const std::vector<int>& order, const std::vector<long long>& cost, int grid) {
+  using Load = std::pair<long long, int>;  // (work so far, CTA): the smallest on top
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < grid; ++c) heap.push({0, c});
+  std::vector<int> owner(order.size()), count(grid, 0);
+  for (size_t i = 0; i < order.size(); ++i) {
+    Load top = heap.top();
+    heap.pop();
+    owner[i] = top.second;
+    ++count[top.second];
+    heap.push({top.first + cost[i], top.second});
+  }
+  L->n = static_cast<int>(order.size());
+  L->start[0] = 0;
+  for (int c = 0; c < grid; ++c) L->start[c + 1] = static_cast<unsigned short>(L->start[c] + count[c]);
+  std::vector<int> fill(L->start, L->start + grid);
+  for (size_t i = 0; i < order.size(); ++i) L->order[fill[owner[i]]++] = static_cast<unsigned short>(order[i]);
+}
+
 bool build_unit_list(fa::FwdUnitList* L, int BH, int N, int d, int bn, int grid) {
   const int NKT = (N + bn - 1) / bn, NQT = (N + 127) / 128, NP = (NQT + 1) / 2, R = 128 / bn;
   const long long units = static_cast<long long>(BH) * NP;
@@ -321,24 +343,13 @@ bool build_unit_list(fa::FwdUnitList* L, int BH, int N, int d, int bn, int grid)
   for (int g0 = 0; g0 < BH; g0 += G)
     for (int r = 0; r < NP; ++r)
       for (int bh = g0; bh < BH && bh < g0 + G; ++bh) order.push_back(r * BH + bh);
-  using Load = std::pair<long long, int>;  // (work so far, CTA): the smallest on top
-  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-  for (int c = 0; c < grid; ++c) heap.push({0, c});
-  std::vector<int> owner(order.size()), count(grid, 0);
+  std::vector<long long> cost(order.size());
   for (size_t i = 0; i < order.size(); ++i) {
     const int qp = NP - 1 - order[i] / BH;
     const int nk0 = std::min((2 * qp + 1) * R, NKT), nk1 = std::min((2 * qp + 2) * R, NKT);
-    Load top = heap.top();
-    heap.pop();
-    owner[i] = top.second;
-    ++count[top.second];
-    heap.push({top.first + nk0 + nk1 + 2 * R, top.second});
+    cost[i] = nk0 + nk1 + 2 * R;
   }
-  L->n = static_cast<int>(order.size());
-  L->start[0] = 0;
-  for (int c = 0; c < grid; ++c) L->start[c + 1] = static_cast<unsigned short>(L->start[c] + count[c]);
-  std::vector<int> fill(L->start, L->start + grid);
-  for (size_t i = 0; i < order.size(); ++i) L->order[fill[owner[i]]++] = static_cast<unsigned short>(order[i]);
+  lpt_assign(L, order, cost, grid);
   return true;
 }
 
@@ -354,6 +365,46 @@ bool causal_unit_list(fa::FwdUnitList* out, int BH, int N, int d, int bn, int gr
   g_lists_next = (g_lists_next + 1) % kListCache;
   e.BH = BH, e.N = N, e.d = d, e.bn = bn, e.grid = grid;
   if (!build_unit_list(&e.list, BH, N, d, bn, grid)) e.list.n = 0;
+  *out = e.list;
+  return e.list.n > 0;
+}
+
+// Unit lists of the persistent fused backward with the mask.  Unit u is key
+// tile kt of head bh in the kernel's grouped order (heads in groups whose K
+// and V fit in 64 MiB of L2, the first key tiles -- those that see the most
+// query tiles -- first); its cost is its query tiles plus one for the unit's
+// fixed work (K and V loads, the dK and dV stores, mostly overlapped).
+UnitListEntry g_bwd_lists[kListCache];
+int g_bwd_lists_next = 0;
+
+bool build_bwd_unit_list(fa::UnitList* L, int BH, int N, int d, int grid) {
+  const int NKT = (N + 127) / 128, NQT = (N + 63) / 64;
+  const long long units = static_cast<long long>(BH) * NKT;
+  if (units > fa::UnitList::kMaxUnits || grid > fa::UnitList::kMaxCtas || grid < 1) return false;
+  const int G = fa::causal_head_group(BH, N, d);
+  std::vector<int> order(units);
+  std::vector<long long> cost(units);
+  for (int u = 0; u < units; ++u) {
+    int bh, kt;
+    fa::causal_grouped_unit(u, BH, NKT, G, bh, kt);
+    order[u] = u;
+    cost[u] = (NQT - (kt * 128) / 64) + 1;
+  }
+  lpt_assign(L, order, cost, grid);
+  return true;
+}
+
+bool causal_bwd_unit_list(fa::UnitList* out, int BH, int N, int d, int grid) {
+  std::lock_guard<std::mutex> lock(g_lists_mu);
+  for (const UnitListEntry& e : g_bwd_lists)
+    if (e.BH == BH && e.N == N && e.d == d && e.grid == grid) {
+      *out = e.list;
+      return e.list.n > 0;
+    }
+  UnitListEntry& e = g_bwd_lists[g_bwd_lists_next];
+  g_bwd_lists_next = (g_bwd_lists_next + 1) % kListCache;
+  e.BH = BH, e.N = N, e.d = d, e.bn = 128, e.grid = grid;
+  if (!build_bwd_unit_list(&e.list, BH, N, d, grid)) e.list.n = 0;
   *out = e.list;
   return e.list.n > 0;
 }
@@ -638,6 +689,11 @@ static int bwd_launch(const void* Q, const void* K, const void* V, const void* O
   };
   const int grid_kv = BH * ((N + 127) / 128);
   const int grid_q = BH * ((N + 127) / 128);
+  // the fused kernel is persistent: one CTA per SM, each walking its units
+  const int grid_fused = grid_kv < sms ? grid_kv : sms;
+  fa::UnitList bul;  // with the mask: this shape's unit lists (n = 0: serpentine deal)
+  bul.n = 0;
+  if (fused && causal) causal_bwd_unit_list(&bul, BH, N, d, grid_fused);
   const unsigned grid_pre = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
   const unsigned grid_cvt = static_cast<unsigned>((rows * d / 8 + 255) / 256);
   mark(0);
@@ -645,8 +701,8 @@ static int bwd_launch(const void* Q, const void* K, const void* V, const void* O
     if (fused) {
       fa::fa_bwd_preprocess_kernel<64, true><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows, dqacc);
       mark(1);
-      if (causal) fa::fa_bwd_fused_kernel<64, true><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
-      else fa::fa_bwd_fused_kernel<64, false><<<grid_kv, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      if (causal) fa::fa_bwd_fused_kernel<64, true><<<grid_fused, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, BH, N, sc, sl2, bul);
+      else fa::fa_bwd_fused_kernel<64, false><<<grid_fused, fa::FusedCfg<64>::THREADS, fa::FusedCfg<64>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, BH, N, sc, sl2, fa::NoUnitList{0});
       mark(2);
       fa::fa_bwd_dq_convert_kernel<<<grid_cvt, 256, 0, s>>>(dqacc, dq, rows * d / 8, sc);
     } else {
@@ -662,8 +718,8 @@ static int bwd_launch(const void* Q, const void* K, const void* V, const void* O
     if (fused) {
       fa::fa_bwd_preprocess_kernel<128, true><<<grid_pre, 256, 0, s>>>(o, dob, Dvec, rows, dqacc);
       mark(1);
-      if (causal) fa::fa_bwd_fused_kernel<128, true><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
-      else fa::fa_bwd_fused_kernel<128, false><<<grid_kv, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, N, sc, sl2);
+      if (causal) fa::fa_bwd_fused_kernel<128, true><<<grid_fused, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, BH, N, sc, sl2, bul);
+      else fa::fa_bwd_fused_kernel<128, false><<<grid_fused, fa::FusedCfg<128>::THREADS, fa::FusedCfg<128>::SMEM_BYTES, s>>>(mqf, mk128, mv128, mdof, LSE, Dvec, dk, dv, dqacc, BH, N, sc, sl2, fa::NoUnitList{0});
       mark(2);
       fa::fa_bwd_dq_convert_kernel<<<grid_cvt, 256, 0, s>>>(dqacc, dq, rows * d / 8, sc);
     } else {

@@ -10,8 +10,8 @@
 //   dV_j = sum_i P_ij dO_i,  dP_ij = dO_i . V_j,  dS_ij = P_ij (dP_ij - D_i)
 //   dK_j = scale sum_i dS_ij Q_i,  dQ_i = scale sum_j dS_ij K_j
 //
-// One CTA per (head, 128-key tile) computes, for every 64-row query tile that
-// can see its keys, all five products: S^T = K Q^T and dP^T = V dO^T into
+// A unit is one (head, 128-key tile); for every 64-row query tile that can
+// see its keys it takes all five products: S^T = K Q^T and dP^T = V dO^T into
 // tensor memory, P^T and dS^T from them, dV += P^T dO and dK += dS^T Q with
 // dV, dK accumulating in tensor memory over the whole loop, and the tile's
 // contribution to dQ, dQ_t^T = K^T dS_t^T (d x 64, fp32).  Every key tile of
@@ -27,10 +27,20 @@
 // are accumulated in a fixed order.  (fa_bwd.cuh holds the deterministic
 // form: a separate dQ kernel that recomputes S and dP, seven products.)
 //
+// The kernel is persistent: one CTA per SM walks its units in order (with
+// the mask, per-CTA lists computed on the host, longest first; otherwise a
+// serpentine deal), so one unit's fixed work overlaps the next one's: its
+// first query tiles load while the previous unit still runs, and its dK and
+// dV are stored while the next unit's K and V load and its first products
+// run.  Every role counts the query tiles of all its units, so the per-tile
+// barriers keep their phases across units.
 // Warp roles (384 threads, three warpgroups):
-//   warp 0       TMA: K and V tiles once; Q and dO tiles through ST stages;
+//   warp 0       TMA: per unit the first ST query tiles (Q and dO, through ST
+//                stages), then K and V once the previous unit's products are
+//                done reading them, then the remaining query tiles;
 //                LSE*log2(e) and D of each query tile into shared memory.
-//   warp 1       tcgen05.mma issue (one elected lane), commits.
+//   warp 1       tcgen05.mma issue (one elected lane), commits; a unit's
+//                first dV and dK wait until the previous unit's are stored.
 //   warps 4-7    softmax gradient: thread = key row.  Reads S^T and dP^T
 //                from tensor memory, writes P^T and dS^T (bf16) back over
 //                S^T's columns (the A operands of dV and dK) and dS^T also to
@@ -42,7 +52,9 @@
 //                d = 64, it reads all 64 columns before staging, so the
 //                tensor-memory buffer returns to the next dP^T product sooner
 //                (measured faster there; without the mask at d = 128 the
-//                smaller register footprint of 32-column steps wins).
+//                smaller register footprint of 32-column steps wins).  After
+//                a unit's last tile: its dK and dV (thread = key row) from
+//                tensor memory to global memory.
 // Tensor memory (512 columns): S^T/P^T/dS^T double buffer [0, 128) (64 each:
 // S^T fp32, then P^T in its first 32 and dS^T in its next 32 columns as packed
 // bf16); dP^T double buffer [128, 256), reused for dQ_t^T once the softmax
@@ -80,26 +92,41 @@ struct FusedCfg {
   static constexpr int OFF_BAR = OFF_DD + ST * BQ * 4;
   static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = 1 + ST, B_S_FULL = 1 + 2 * ST,
                        B_P_FULL = B_S_FULL + 2, B_DQ_FULL = B_P_FULL + 2, B_DQ_EMPTY = B_DQ_FULL + 2,
-                       B_STG_FREE = B_DQ_EMPTY + 2, B_STG_FULL = B_STG_FREE + NDQ, B_DKV_FULL = B_STG_FULL + NDQ;
-  static constexpr int NUM_BARS = B_DKV_FULL + 1;
+                       B_STG_FREE = B_DQ_EMPTY + 2, B_STG_FULL = B_STG_FREE + NDQ, B_DKV_FULL = B_STG_FULL + NDQ,
+                       B_KV_EMPTY = B_DKV_FULL + 1, B_ACC_EMPTY = B_KV_EMPTY + 1;
+  static constexpr int NUM_BARS = B_ACC_EMPTY + 1;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;  // + room to align the base to 1024
   static_assert(SMEM_BYTES <= 232448, "shared memory of the fused backward exceeds 227 KB");
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
-  // register split (launch: 384 x 168 = 64512): control 64 and dQ drain 160
+  // register split (launch: 384 x 168 = 64512): control 112 and dQ drain 136
   // (both decrease: never above the 168 of the launch), softmax gradient 256
-  // (128 x 480 = 61440)
-  static constexpr uint32_t REGS_CONTROL = 64, REGS_GRAD = 256, REGS_DRAIN = 160;
+  // (128 x 504 = 64512)
+  static constexpr uint32_t REGS_CONTROL = 112, REGS_GRAD = 256, REGS_DRAIN = 136;
   static_assert(REGS_CONTROL <= 168 && REGS_DRAIN <= 168 && 128 * (REGS_CONTROL + REGS_GRAD + REGS_DRAIN) <= 64512,
                 "register split must fit the registers of the launch");
 };
 
 enum FusedWaitSite : unsigned int {
   BF_PROD_QE = 64, BF_MMA_KV, BF_MMA_Q, BF_MMA_DQE, BF_MMA_P, BF_SM_S, BF_SM_Q, BF_SM_DKV, BF_DR_DQ, BF_DR_FREE,
-  BF_DR_FULL
+  BF_DR_FULL, BF_PROD_KVE, BF_MMA_ACC
 };
+
+// Unit u of the persistent kernel: key tile kt of head bh.  Without the mask
+// head-major (the CTAs running at the same time share a few heads' Q and dO
+// in L2); with it, the longest key tiles (the first ones) of every head of an
+// L2-sized group first (the host's lists assign them longest first).
+template <bool CAUSAL>
+__device__ __forceinline__ void fused_unit(int u, int BH, int NKT, int N, int D, int& bh, int& kt) {
+  if (CAUSAL) {
+    causal_grouped_unit(u, BH, NKT, causal_head_group(BH, N, D), bh, kt);
+  } else {
+    bh = u / NKT;
+    kt = u - bh * NKT;
+  }
+}
 
 // Query tile of the it-th step of key tile kt.  With the mask the steps start
 // at the first query tile that sees the keys (i0) and walk up.  Without it
@@ -114,13 +141,39 @@ __device__ __forceinline__ int fused_query_tile(int it, int i0, int nt, int kt) 
   return q;
 }
 
+// One row of an accumulator (dK or dV: this thread's tensor-memory lane) to
+// global memory as bf16, times `mul`: D/32 loads of 32 columns, 16-byte stores.
+template <int D>
+__device__ __forceinline__ void store_accumulator_row(uint32_t t_row, __nv_bfloat16* dst_row, float mul, bool valid) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t a[32];
+    tmem_ld32(t_row + cc * 32, a);
+    tmem_ld_wait();
+    reg_fence(a);
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 wv;
+        wv.x = pack_bf16(__uint_as_float(a[8 * v + 0]) * mul, __uint_as_float(a[8 * v + 1]) * mul);
+        wv.y = pack_bf16(__uint_as_float(a[8 * v + 2]) * mul, __uint_as_float(a[8 * v + 3]) * mul);
+        wv.z = pack_bf16(__uint_as_float(a[8 * v + 4]) * mul, __uint_as_float(a[8 * v + 5]) * mul);
+        wv.w = pack_bf16(__uint_as_float(a[8 * v + 6]) * mul, __uint_as_float(a[8 * v + 7]) * mul);
+        dst[v] = wv;
+      }
+    }
+  }
+}
+
 template <int D, bool CAUSAL, int ST_ = ((D == 128) ? 3 : 4), int NDQ_ = ((D == 128) ? 1 : 2)>
 __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
     fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                         const float* __restrict__ LSE, const float* __restrict__ Dvec,
                         __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
-                        float* __restrict__ dQacc, int N, float scale, float scale_log2) {
+                        float* __restrict__ dQacc, int BH, int N, float scale, float scale_log2,
+                        const __grid_constant__ typename UnitListOf<CAUSAL>::type list) {
   using C = FusedCfg<D, ST_, NDQ_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -133,20 +186,16 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Block order: head-major without the mask; with it, the longest key tiles
-  // (the first ones) of every head of an L2-sized group first.
+  // Persistent: this CTA walks its units (key tiles of heads) in order; every
+  // role counts the query tiles of the units before the current one (tb), so
+  // the per-tile barriers keep their phases across units.
   const int NKT = (N + C::BK - 1) / C::BK;
-  const int BHg = gridDim.x / NKT;
-  int bh, kt;
-  if (CAUSAL) {
-    causal_grouped_unit(blockIdx.x, BHg, NKT, causal_head_group(BHg, N, D), bh, kt);
-  } else {
-    bh = blockIdx.x / NKT;
-    kt = blockIdx.x - bh * NKT;
-  }
   const int NQT = (N + C::BQ - 1) / C::BQ;
-  const int i0 = CAUSAL ? (kt * C::BK) / C::BQ : 0;
-  const int nt = NQT - i0;  // >= 1
+  const int units = BH * NKT;
+  auto unit_tiles = [&](int kt, int& i0, int& nt) {
+    i0 = CAUSAL ? (kt * C::BK) / C::BQ : 0;
+    nt = NQT - i0;  // >= 1
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bars + 8 * C::B_KV_FULL, 1);
@@ -165,6 +214,8 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       mbar_init(bars + 8 * (C::B_STG_FULL + b), 128);  // every drain thread: its column is stored
     }
     mbar_init(bars + 8 * C::B_DKV_FULL, 1);
+    mbar_init(bars + 8 * C::B_KV_EMPTY, 1);    // the unit's last product that reads K and V is done
+    mbar_init(bars + 8 * C::B_ACC_EMPTY, 128);  // the drain warps have stored the unit's dK and dV
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -183,34 +234,56 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmdO);
-        mbar_arrive_expect_tx(bars + 8 * C::B_KV_FULL, 2 * C::K_TILE);
-        for (int c = 0; c < C::CH; ++c) {
-          tma_load_3d(sK + c * C::KCHUNK, &tmK, bars + 8 * C::B_KV_FULL, c * 64, kt * C::BK, bh);
-          tma_load_3d(sV + c * C::KCHUNK, &tmV, bars + 8 * C::B_KV_FULL, c * 64, kt * C::BK, bh);
-        }
       }
-      for (int it = 0; it < nt; ++it) {
-        const int st = it % C::ST;
-        const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
-        const bool ok = mbar_wait(bars + 8 * (C::B_Q_EMPTY + st), ((it / C::ST) & 1) ^ 1, BF_PROD_QE);
-        if (!__all_sync(0xffffffffu, ok)) break;
+      int tb = 0;
+      bool ok = true;
+      for (int k = 0, u = list_unit(list, 0, units); u < units && ok; u = list_unit(list, ++k, units)) {
+        int bh, kt, i0, nt;
+        fused_unit<CAUSAL>(u, BH, NKT, N, D, bh, kt);
+        unit_tiles(kt, i0, nt);
+        // query tile it of this unit into its stage (once the tile that used the
+        // stage before has had its dV and dK products)
+        auto load_q = [&](int it) -> bool {
+          const int g = tb + it, st = g % C::ST;
+          const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
+          if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_EMPTY + st), ((g / C::ST) & 1) ^ 1, BF_PROD_QE)))
+            return false;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bars + 8 * (C::B_Q_FULL + st), 2 * C::Q_TILE);
+            for (int c = 0; c < C::CH; ++c) {
+              tma_load_3d(sQ + st * C::Q_TILE + c * C::QCHUNK, &tmQ, bars + 8 * (C::B_Q_FULL + st), c * 64,
+                          qi * C::BQ, bh);
+              tma_load_3d(sdO + st * C::Q_TILE + c * C::QCHUNK, &tmdO, bars + 8 * (C::B_Q_FULL + st), c * 64,
+                          qi * C::BQ, bh);
+            }
+          }
+#pragma unroll
+          for (int e = lane; e < C::BQ; e += 32) {
+            const int q = qi * C::BQ + e;
+            const bool valid = q < N;
+            sLSE[st * C::BQ + e] = valid ? LSE[static_cast<size_t>(bh) * N + q] * kLog2e : INFINITY;
+            sDD[st * C::BQ + e] = valid ? Dvec[static_cast<size_t>(bh) * N + q] : 0.f;
+          }
+          mbar_arrive(bars + 8 * (C::B_Q_FULL + st));
+          return true;
+        };
+        // the unit's first query tiles go while the previous unit still runs;
+        // K and V once the previous unit's products are done reading them
+        const int early = nt < C::ST ? nt : C::ST;
+        for (int it = 0; it < early && ok; ++it) ok = load_q(it);
+        if (!ok) break;
+        if (k > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_KV_EMPTY, (k - 1) & 1, BF_PROD_KVE))))
+          break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(bars + 8 * (C::B_Q_FULL + st), 2 * C::Q_TILE);
+          mbar_arrive_expect_tx(bars + 8 * C::B_KV_FULL, 2 * C::K_TILE);
           for (int c = 0; c < C::CH; ++c) {
-            tma_load_3d(sQ + st * C::Q_TILE + c * C::QCHUNK, &tmQ, bars + 8 * (C::B_Q_FULL + st), c * 64,
-                        qi * C::BQ, bh);
-            tma_load_3d(sdO + st * C::Q_TILE + c * C::QCHUNK, &tmdO, bars + 8 * (C::B_Q_FULL + st), c * 64,
-                        qi * C::BQ, bh);
+            tma_load_3d(sK + c * C::KCHUNK, &tmK, bars + 8 * C::B_KV_FULL, c * 64, kt * C::BK, bh);
+            tma_load_3d(sV + c * C::KCHUNK, &tmV, bars + 8 * C::B_KV_FULL, c * 64, kt * C::BK, bh);
           }
         }
-#pragma unroll
-        for (int e = lane; e < C::BQ; e += 32) {
-          const int q = qi * C::BQ + e;
-          const bool valid = q < N;
-          sLSE[st * C::BQ + e] = valid ? LSE[static_cast<size_t>(bh) * N + q] * kLog2e : INFINITY;
-          sDD[st * C::BQ + e] = valid ? Dvec[static_cast<size_t>(bh) * N + q] : 0.f;
-        }
-        mbar_arrive(bars + 8 * (C::B_Q_FULL + st));
+        for (int it = early; it < nt && ok; ++it) ok = load_q(it);
+        if (!ok) break;
+        tb += nt;
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issue (whole warp, one elected lane)
@@ -234,53 +307,73 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       // 64-column chunks KCHUNK apart; at d = 64 the second chunk is the V
       // tile), B = dS^T read MN-major (N = 64 queries, one chunk); K = 128 keys.
       const uint64_t dq_a = sdesc_make(sdesc_lo(sK, C::KCHUNK), sdesc_hi(1024));
-      bool ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_KV_FULL, 0, BF_MMA_KV));
-      tc_fence_after();
-      for (int it = 0; it <= nt && ok; ++it) {
-        if (it < nt) {
-          const int st = it % C::ST, b = it & 1;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_FULL + st), (it / C::ST) & 1, BF_MMA_Q))))
-            break;
-          tc_fence_after();
-          issue_t(tmem + C::TM_S + b * 64, sK, sQ + st * C::Q_TILE);
-          if (it >= 2) {  // dP^T's buffer holds dQ^T of tile it-2 until the drain has read it
-            if (!(ok = __all_sync(0xffffffffu,
-                                  mbar_wait(bars + 8 * (C::B_DQ_EMPTY + b), ((it >> 1) & 1) ^ 1, BF_MMA_DQE))))
+      int tb = 0;
+      bool ok = true;
+      for (int k = 0, u = list_unit(list, 0, units); u < units && ok; u = list_unit(list, ++k, units)) {
+        int bh, kt, i0, nt;
+        fused_unit<CAUSAL>(u, BH, NKT, N, D, bh, kt);
+        unit_tiles(kt, i0, nt);
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_KV_FULL, k & 1, BF_MMA_KV)))) break;
+        tc_fence_after();
+        for (int it = 0; it <= nt && ok; ++it) {
+          if (it < nt) {
+            const int g = tb + it, st = g % C::ST, b = g & 1;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_FULL + st), (g / C::ST) & 1, BF_MMA_Q))))
               break;
             tc_fence_after();
+            issue_t(tmem + C::TM_S + b * 64, sK, sQ + st * C::Q_TILE);
+            if (g >= 2) {  // dP^T's buffer holds dQ^T of tile g-2 until the drain has read it
+              if (!(ok = __all_sync(0xffffffffu,
+                                    mbar_wait(bars + 8 * (C::B_DQ_EMPTY + b), ((g >> 1) & 1) ^ 1, BF_MMA_DQE))))
+                break;
+              tc_fence_after();
+            }
+            issue_t(tmem + C::TM_DP + b * 64, sV, sdO + st * C::Q_TILE);
+            tc_commit_warp(bars + 8 * (C::B_S_FULL + b));
           }
-          issue_t(tmem + C::TM_DP + b * 64, sV, sdO + st * C::Q_TILE);
-          tc_commit_warp(bars + 8 * (C::B_S_FULL + b));
+          if (it > 0) {
+            const int pit = it - 1, pg = tb + pit, pst = pg % C::ST, pb = pg & 1;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pg >> 1) & 1, BF_MMA_P))))
+              break;
+            // the unit's first dV and dK overwrite the accumulators: the drain
+            // warps must have read the previous unit's
+            if (pit == 0 && k > 0 &&
+                !(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_ACC_EMPTY, (k - 1) & 1, BF_MMA_ACC))))
+              break;
+            tc_fence_after();
+            issue_g(tmem + C::TM_DV, tmem + C::TM_S + pb * 64, sdO + pst * C::Q_TILE, pit > 0);
+            issue_g(tmem + C::TM_DK, tmem + C::TM_S + pb * 64 + 32, sQ + pst * C::Q_TILE, pit > 0);
+            tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + pst));
+            mma_ss_k128_mnmn(tmem + C::TM_DP + pb * 64, dq_a,
+                             sdesc_make(sdesc_lo(sDS + pb * C::DS_TILE, C::DS_TILE), sdesc_hi(1024)), IDESC_DQ, 0u);
+            tc_commit_warp(bars + 8 * (C::B_DQ_FULL + pb));
+          }
         }
-        if (it > 0) {
-          const int pit = it - 1, pst = pit % C::ST, pb = pit & 1;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_P_FULL + pb), (pit >> 1) & 1, BF_MMA_P))))
-            break;
-          tc_fence_after();
-          issue_g(tmem + C::TM_DV, tmem + C::TM_S + pb * 64, sdO + pst * C::Q_TILE, pit > 0);
-          issue_g(tmem + C::TM_DK, tmem + C::TM_S + pb * 64 + 32, sQ + pst * C::Q_TILE, pit > 0);
-          tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + pst));
-          mma_ss_k128_mnmn(tmem + C::TM_DP + pb * 64, dq_a,
-                           sdesc_make(sdesc_lo(sDS + pb * C::DS_TILE, C::DS_TILE), sdesc_hi(1024)), IDESC_DQ, 0u);
-          tc_commit_warp(bars + 8 * (C::B_DQ_FULL + pb));
-        }
+        if (!ok) break;
+        tc_commit_warp(bars + 8 * C::B_KV_EMPTY);  // K and V free for the next unit's loads
+        tc_commit_warp(bars + 8 * C::B_DKV_FULL);  // dK and dV complete
+        tb += nt;
       }
-      if (ok) tc_commit_warp(bars + 8 * C::B_DKV_FULL);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax gradient (thread = key row)
     regs_inc<C::REGS_GRAD>();
     const int sp = warp & 3;
     const int r = sp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
+    int tb = 0;
+    bool ok = true;
+    for (int k = 0, u = list_unit(list, 0, units); u < units && ok; u = list_unit(list, ++k, units)) {
+    int bh, kt, i0, nt;
+    fused_unit<CAUSAL>(u, BH, NKT, N, D, bh, kt);
+    unit_tiles(kt, i0, nt);
     const int key = kt * C::BK + r;
     const bool key_valid = key < N;
-    const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
-    bool ok = true;
-    for (int it = 0; it < nt; ++it) {
-      const int st = it % C::ST, b = it & 1;
-      const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
-      bool w = mbar_wait(bars + 8 * (C::B_S_FULL + b), (it >> 1) & 1, BF_SM_S);
-      w = w && mbar_wait(bars + 8 * (C::B_Q_FULL + st), (it / C::ST) & 1, BF_SM_Q);
+    int qi = fused_query_tile<CAUSAL>(0, i0, nt, kt);  // advanced by one (mod NQT) per tile
+    for (int it = 0; it < nt; ++it, qi = qi + 1 == NQT ? 0 : qi + 1) {
+      const int g = tb + it, st = g % C::ST, b = g & 1;
+      bool w = mbar_wait(bars + 8 * (C::B_S_FULL + b), (g >> 1) & 1, BF_SM_S);
+      w = w && mbar_wait(bars + 8 * (C::B_Q_FULL + st), (g / C::ST) & 1, BF_SM_Q);
       if (!(ok = __all_sync(0xffffffffu, w))) break;
       tc_fence_after();
       const uint32_t tS = tmem + lane_off + C::TM_S + b * 64;
@@ -340,34 +433,7 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       tc_fence_before();
       mbar_arrive(bars + 8 * (C::B_P_FULL + b));
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_DKV_FULL, 0, BF_SM_DKV))) {
-      tc_fence_after();
-      const size_t base = (static_cast<size_t>(bh) * N + key) * D;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tA = tmem + lane_off + (which ? C::TM_DK : C::TM_DV);
-        __nv_bfloat16* dst_row = (which ? dK : dV) + base;
-        const float mul = which ? scale : 1.f;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t a[32];
-          tmem_ld32(tA + c * 32, a);
-          tmem_ld_wait();
-          reg_fence(a);
-          if (key_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 wv;
-              wv.x = pack_bf16(__uint_as_float(a[8 * v + 0]) * mul, __uint_as_float(a[8 * v + 1]) * mul);
-              wv.y = pack_bf16(__uint_as_float(a[8 * v + 2]) * mul, __uint_as_float(a[8 * v + 3]) * mul);
-              wv.z = pack_bf16(__uint_as_float(a[8 * v + 4]) * mul, __uint_as_float(a[8 * v + 5]) * mul);
-              wv.w = pack_bf16(__uint_as_float(a[8 * v + 6]) * mul, __uint_as_float(a[8 * v + 7]) * mul);
-              dst[v] = wv;
-            }
-          }
-        }
-      }
+    tb += nt;
     }
   } else {
     // ------------------------------------------------------------ dQ drain (thread = column c of d)
@@ -378,10 +444,16 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(sp * 32) << 16;
     const bool issuer = threadIdx.x == 256;
     float* stg = reinterpret_cast<float*>(smem + C::OFF_DQ);
+    int tb = 0;
+    bool ok = true;
+    for (int k = 0, u = list_unit(list, 0, units); u < units && ok; u = list_unit(list, ++k, units)) {
+    int bh, kt, i0, nt;
+    fused_unit<CAUSAL>(u, BH, NKT, N, D, bh, kt);
+    unit_tiles(kt, i0, nt);
     for (int it = 0; it < nt; ++it) {
-      const int b = it & 1, sb = it % C::NDQ;
+      const int g = tb + it, b = g & 1, sb = g % C::NDQ;
       const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
-      if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_DQ_FULL + b), (it >> 1) & 1, BF_DR_DQ))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_DQ_FULL + b), (g >> 1) & 1, BF_DR_DQ)))) break;
       tc_fence_after();
       if constexpr (CAUSAL || D == 64) {
         // all 64 columns into registers, release the tensor-memory buffer at
@@ -401,7 +473,7 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
           bulk_wait_read<C::NDQ - 1>();
           mbar_arrive(bars + 8 * (C::B_STG_FREE + sb));
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (it / C::NDQ) & 1, BF_DR_FREE)))
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (g / C::NDQ) & 1, BF_DR_FREE))))
           break;
         if (active) {
           float* t = stg + sb * (C::DQ_TILE / 4) + c;
@@ -415,7 +487,7 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
           bulk_wait_read<C::NDQ - 1>();
           mbar_arrive(bars + 8 * (C::B_STG_FREE + sb));
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (it / C::NDQ) & 1, BF_DR_FREE)))
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (g / C::NDQ) & 1, BF_DR_FREE))))
           break;
         if (active) {
           float* t = stg + sb * (C::DQ_TILE / 4) + c;
@@ -436,7 +508,7 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       mbar_arrive(bars + 8 * (C::B_STG_FULL + sb));
       bool stored = true;
       if (issuer) {
-        stored = mbar_wait(bars + 8 * (C::B_STG_FULL + sb), (it / C::NDQ) & 1, BF_DR_FULL);
+        stored = mbar_wait(bars + 8 * (C::B_STG_FULL + sb), (g / C::NDQ) & 1, BF_DR_FULL);
         if (stored) {
           const int rows = min(C::BQ, N - qi * C::BQ);
           bulk_reduce_add_f32(dQacc + (static_cast<size_t>(bh) * N + static_cast<size_t>(qi) * C::BQ) * D,
@@ -444,7 +516,22 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
           bulk_commit();
         }
       }
-      if (!__all_sync(0xffffffffu, stored)) break;
+      if (!(ok = __all_sync(0xffffffffu, stored))) break;
+    }
+    if (!ok) break;
+    // the unit's dK and dV (thread = key row of the warp's lane window), while
+    // the next unit's K and V load and the softmax warps start on its tiles
+    if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * C::B_DKV_FULL, k & 1, BF_SM_DKV)))) break;
+    tc_fence_after();
+    {
+      const int key = kt * C::BK + sp * 32 + lane;
+      const size_t row = (static_cast<size_t>(bh) * N + key) * D;
+      store_accumulator_row<D>(tmem + lane_off + C::TM_DV, dV + row, 1.f, key < N);
+      store_accumulator_row<D>(tmem + lane_off + C::TM_DK, dK + row, scale, key < N);
+    }
+    tc_fence_before();
+    mbar_arrive(bars + 8 * C::B_ACC_EMPTY);
+    tb += nt;
     }
     if (issuer) bulk_wait_all();
   }
@@ -456,6 +543,7 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
+
 
 // ---------------------------------------------------------------------------
 // dQ = bf16(scale * accumulator): eight elements per thread, 16-byte stores

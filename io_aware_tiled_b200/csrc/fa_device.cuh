@@ -692,20 +692,55 @@ __device__ __forceinline__ int serpentine_unit(int k, int w, int W) {
 // V (or Q and dO) in flight.  Heads therefore go in groups whose K and V
 // (bf16) fit in 64 MiB of the 126 MB L2 (all heads when they fit), longest
 // blocks first inside each group.  Returns the group size.
-__device__ __forceinline__ int causal_head_group(int BH, int N, int D) {
+__host__ __device__ __forceinline__ int causal_head_group(int BH, int N, int D) {
   const long long per_head = 4ll * N * D;
   const long long g = (64ll << 20) / per_head;
   return g >= BH ? BH : (g < 1 ? 1 : static_cast<int>(g));
 }
 // Unit u of that order for units of NR ranks per head (rank 0 = longest):
 // head bh and rank r.
-__device__ __forceinline__ void causal_grouped_unit(int u, int BH, int NR, int G, int& bh, int& r) {
+__host__ __device__ __forceinline__ void causal_grouped_unit(int u, int BH, int NR, int G, int& bh, int& r) {
   const int per_group = G * NR;
   const int g = u / per_group;
   const int v = u - g * per_group;
-  const int gh = min(G, BH - g * G);  // heads in this group (the last may be short)
+  const int gh = G < BH - g * G ? G : BH - g * G;  // heads in this group (the last may be short)
   r = v / gh;
   bh = g * G + (v - r * gh);
+}
+
+// Per-CTA work lists of the persistent kernels, computed on the host (a
+// longest-processing-time assignment) and passed by value: CTA c runs the
+// units order[start[c] .. start[c + 1]) in that order.  n = 0: no list.
+struct UnitList {
+  static constexpr int kMaxCtas = 160;
+  static constexpr int kMaxUnits = 4096;
+  int n;                                   // units in `order`
+  unsigned short start[kMaxCtas + 1];
+  unsigned short order[kMaxUnits];         // unit indices, in each kernel's own numbering
+};
+struct NoUnitList {
+  int n;
+};
+template <bool WITH_LIST>
+struct UnitListOf {
+  using type = NoUnitList;
+};
+template <>
+struct UnitListOf<true> {
+  using type = UnitList;
+};
+
+// The k-th unit of this CTA in `list` (>= units when it has no more); without
+// a list, the units dealt in serpentine order over the grid.
+template <typename L>
+__device__ __forceinline__ int list_unit(const L& list, int k, int units) {
+  if constexpr (sizeof(L) > sizeof(NoUnitList)) {
+    if (list.n > 0) {
+      const int i = list.start[blockIdx.x] + k;
+      return i < list.start[blockIdx.x + 1] ? static_cast<int>(list.order[i]) : units;
+    }
+  }
+  return serpentine_unit(k, blockIdx.x, gridDim.x);
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -132,38 +132,17 @@ __device__ __forceinline__ void ring_tile(int i, int nk0, int& j, int& t) {
   }
 }
 
-// Per-CTA unit lists of the causal forward, computed on the host (a
-// longest-processing-time assignment over an L2-friendly unit order) and
-// passed by value.  n = 0: no list; the units are dealt in serpentine order.
-struct FwdUnitList {
-  static constexpr int kMaxCtas = 160;
-  static constexpr int kMaxUnits = 4096;
-  int n;                                   // units in `order`
-  unsigned short start[kMaxCtas + 1];      // CTA c takes order[start[c] .. start[c + 1])
-  unsigned short order[kMaxUnits];         // unit indices as fwd_decode_unit reads them
-};
-struct FwdNoList {
-  int n;
-};
+// Per-CTA unit lists of the causal forward (UnitList): unit indices as
+// fwd_decode_unit reads them; none without the mask.
+using FwdUnitList = UnitList;
+using FwdNoList = NoUnitList;
 template <bool CAUSAL>
-struct FwdListOf {
-  using type = FwdNoList;
-};
-template <>
-struct FwdListOf<true> {
-  using type = FwdUnitList;
-};
+using FwdListOf = UnitListOf<CAUSAL>;
 
 // The k-th unit of this CTA (>= units when it has no more).
 template <typename L>
 __device__ __forceinline__ int fwd_unit(const L& list, int k, int units) {
-  if constexpr (sizeof(L) > sizeof(FwdNoList)) {
-    if (list.n > 0) {
-      const int i = list.start[blockIdx.x] + k;
-      return i < list.start[blockIdx.x + 1] ? static_cast<int>(list.order[i]) : units;
-    }
-  }
-  return serpentine_unit(k, blockIdx.x, gridDim.x);
+  return list_unit(list, k, units);
 }
 
 template <int D, bool CAUSAL, int BN_ = 128>

@@ -337,6 +337,32 @@ def test_fused_and_deterministic_backward_agree(B, H, N, d):
                 assert_same_up_to_summation_order(a, b, name + " " + what)
 
 
+def test_persistent_backward_walks_every_unit():
+    """The default backward's kernel is persistent: one CTA per SM walks its
+    key-tile units (lists computed on the host with the mask, at most 4096
+    units; beyond that, and without the mask, a serpentine deal).  Shapes
+    with one unit per CTA, many units per CTA and more units than the lists
+    hold all give the deterministic form's dK and dV bit for bit with the mask
+    (the same products in the same order) and dQ up to summation order."""
+    dev = _dev()
+    for B, H, N, d, causals in ((1, 1, 130, 64, (False, True)),        # 2 units, fewer than the SMs
+                                (2, 8, 1280, 128, (False, True)),      # 160 units: some CTAs take two
+                                (4, 300, 1024, 64, (True,))):          # 9600 units: past the lists
+        q, k, v, do = (t.to(dev) for t in attention_inputs(B, H, N, d, seed=31 + N))
+        for causal in causals:
+            o, lse = fa.forward(q, k, v, causal)
+            fu = fa.backward(q, k, v, o, do, lse, causal)
+            de = fa.backward(q, k, v, o, do, lse, causal, deterministic=True)
+            assert fa.sync_status() == fa.FA_OK
+            what = f"{B,H,N,d} causal={causal}"
+            assert_same_up_to_summation_order(fu[0], de[0], "dQ " + what)
+            for name, a, b in (("dK", fu[1], de[1]), ("dV", fu[2], de[2])):
+                if causal:
+                    assert torch.equal(a, b), name + " " + what
+                else:
+                    assert_same_up_to_summation_order(a, b, name + " " + what)
+
+
 def test_autograd_wrapper_runs_library_kernels():
     dev = _dev()
     q, k, v, do = attention_inputs(1, 2, 256, 64, seed=12)
