@@ -322,6 +322,8 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
             if (i + C::NS < n) ok = s_of(i + C::NS);
           }
           if (!ok) break;
+          // (two Q pairs: the next unit's is already loaded, so the release
+          // can wait for the unit's end)
           tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));
           kv_it += nk1;
           g0 += n;
@@ -349,6 +351,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           issue_s(tmem + C::TM_S1, sQb + C::Q_TILE, sK + s * C::KV_TILE);
           tc_commit_warp(bars + 8 * (C::B_S_FULL + 1));
           tc_commit_warp(bars + 8 * (C::B_K_EMPTY + s));
+          if (nk1 == 1) tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));  // no further S reads the Q pair
         }
         for (int j = 0; j < nk1 && ok; ++j) {
           const uint32_t it = kv_it + j;
@@ -385,15 +388,19 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
             issue_s(tmem + C::TM_S1, sQb + C::Q_TILE, sK + sn * C::KV_TILE);
             tc_commit_warp(bars + 8 * (C::B_S_FULL + 1));
             tc_commit_warp(bars + 8 * (C::B_K_EMPTY + sn));
+            // the unit's last S: its Q pair is free for the next unit's loads
+            // (the PVs still to come do not read Q)
+            if (j + 2 == nk1) tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));
           }
         }
         if (!ok) break;
-        tc_commit_warp(bars + 8 * (C::B_Q_EMPTY + qb));
         kv_it += nk1;
       }
       }
-      // The last unit's Q_EMPTY arrival is the last one this thread's commits
-      // make; wait for it so no arrival lands after the CTA has exited.
+      // Wait for the last unit's Q_EMPTY arrival, so none lands after the CTA
+      // has exited: with the S ring it is this thread's last commit; with two
+      // S buffers it precedes the last PV's commits, whose final O_FULL
+      // arrival the softmax warpgroups wait for before the teardown.
       if (q_it > 0)
         (void)__all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_Q_EMPTY + (q_it - 1) % C::NQB),
                                                 ((q_it - 1) / C::NQB) & 1, FW_MMA_Q));

@@ -211,7 +211,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
       ++q_it;
       tc_fence_after();
       const uint32_t s_base = s_it;  // buffer of this unit's tile j is (s_base + j) % NS
-      for (int j = 0; j < nk && j < C::NS && ok; ++j) ok = issue_s(kv_it + j, (s_base + j) % C::NS);
+      // after the unit's last S its Q half is free for the next unit's loads
+      // (the PVs still to come do not read Q)
+      for (int j = 0; j < nk && j < C::NS && ok; ++j) {
+        ok = issue_s(kv_it + j, (s_base + j) % C::NS);
+        if (ok && j == nk - 1) tc_commit_pair_warp(bar(C::B_Q_EMPTY), C::BOTH);
+      }
       for (int j = 0; j < nk && ok; ++j) {
         const uint32_t it = kv_it + j;
         const int s = it % C::ST, b = (s_base + j) % C::NS;
@@ -228,16 +233,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
                      IDESC_PV, j > 0 ? 1u : 0u);
         tc_commit_pair_warp(bar(C::B_O_DONE + ((s_base + j) & 1)), C::BOTH);
         tc_commit_pair_warp(bar(C::B_V_EMPTY + s), C::BOTH);
-        if (j + C::NS < nk) ok = issue_s(it + C::NS, b);  // buffer b is free once PV_j has read P_j
+        if (j + C::NS < nk) {
+          ok = issue_s(it + C::NS, b);  // buffer b is free once PV_j has read P_j
+          if (ok && j + C::NS == nk - 1) tc_commit_pair_warp(bar(C::B_Q_EMPTY), C::BOTH);
+        }
       }
       if (!ok) break;
-      tc_commit_pair_warp(bar(C::B_Q_EMPTY), C::BOTH);
       kv_it += nk;
       s_it += nk;
     }
-    // The last unit's Q_EMPTY arrival is the last one the commits make.
-    if (ok && q_it > 0)
-      (void)__all_sync(0xffffffffu, mbar_wait_cluster(bar(C::B_Q_EMPTY), (q_it - 1) & 1, F2_MMA_Q));
+    // The last PV's V_EMPTY arrival is the last one the commits make (the
+    // unit's Q_EMPTY went out after its last S); wait for it here, so none
+    // lands after the teardown.
+    if (ok && kv_it > 0)
+      (void)__all_sync(0xffffffffu, mbar_wait_cluster(bar(C::B_V_EMPTY + (kv_it - 1) % C::ST),
+                                                     ((kv_it - 1) / C::ST) & 1, F2_MMA_V));
   } else if (warp == 1) {
     // ------------------------------------------------------------ relay (CTA 1)
     // Forwards each completed phase of CTA 1's P and O-empty barriers to the
