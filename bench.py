@@ -305,9 +305,9 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
     # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal_dram.md (32 heads)
-    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.752384e6 + 14.939648e6) / 32,
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.752896e6 + 14.989056e6) / 32,
                           "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "c52a3cf30de8f792f7d37983e698cad59d208f19b31f5e571dfd88d3011714cf"},
+                          "sha256": "f428f9dfcfe88488595cb49ee7e0cda682e39970c17846694a8c9bfe4cdb5b5b"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
     "fa_bwd_fused_kernel": {"bytes_per_head": (202.848256e6 + 85.483776e6) / 32,
