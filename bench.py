@@ -310,9 +310,9 @@ NCU_TRAFFIC = {
                           "sha256": "f428f9dfcfe88488595cb49ee7e0cda682e39970c17846694a8c9bfe4cdb5b5b"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
-    "fa_bwd_fused_kernel": {"bytes_per_head": (202.848256e6 + 85.483776e6) / 32,
+    "fa_bwd_fused_kernel": {"bytes_per_head": (202.483968e6 + 84.928e6) / 32,
                             "sources": ("fa_bwd_fused.cuh", "fa_device.cuh"),
-                            "sha256": "6dcc818fafe19c681afbcb02cf6c9b2353c6bbdc8702fbd8717d313396218810"},
+                            "sha256": "105bf34fac7f3c4da0ff73015c2bd47077d6590b103b4b4fd380f32faddc2c1f"},
 }
 
 

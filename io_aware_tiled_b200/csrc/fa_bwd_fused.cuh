@@ -48,11 +48,9 @@
 //   warps 8-11   dQ drain: thread = column c of d.  Reads dQ_t^T from tensor
 //                memory, stores it as a [64 queries][d] fp32 tile in shared
 //                memory and issues the bulk reduce-add of that tile into the
-//                accumulator rows of the query tile.  With the mask, and at
-//                d = 64, it reads all 64 columns before staging, so the
-//                tensor-memory buffer returns to the next dP^T product sooner
-//                (measured faster there; without the mask at d = 128 the
-//                smaller register footprint of 32-column steps wins).  After
+//                accumulator rows of the query tile.  It reads all 64
+//                columns into registers before staging, so the tensor-memory
+//                buffer returns to the next dP^T product sooner.  After
 //                a unit's last tile: its dK and dV (thread = key row) from
 //                tensor memory to global memory.
 // Tensor memory (512 columns): S^T/P^T/dS^T double buffer [0, 128) (64 each:
@@ -455,54 +453,29 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       const int qi = fused_query_tile<CAUSAL>(it, i0, nt, kt);
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_DQ_FULL + b), (g >> 1) & 1, BF_DR_DQ)))) break;
       tc_fence_after();
-      if constexpr (CAUSAL || D == 64) {
-        // all 64 columns into registers, release the tensor-memory buffer at
-        // once (the next dP^T product may go ahead), then stage
-        uint32_t v[64];
-        if (active) {
-          tmem_ld32(tmem + lane_off + C::TM_DP + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          tmem_ld32(tmem + lane_off + C::TM_DP + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-          tmem_ld_wait();
-          reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        }
-        tc_fence_before();
-        mbar_arrive(bars + 8 * (C::B_DQ_EMPTY + b));
-        // the staging buffer sb is free once the reduce issued NDQ tiles ago has read it
-        if (issuer) {
-          bulk_wait_read<C::NDQ - 1>();
-          mbar_arrive(bars + 8 * (C::B_STG_FREE + sb));
-        }
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (g / C::NDQ) & 1, BF_DR_FREE))))
-          break;
-        if (active) {
-          float* t = stg + sb * (C::DQ_TILE / 4) + c;
+      // all 64 columns into registers, release the tensor-memory buffer at
+      // once (the next dP^T product may go ahead), then stage
+      uint32_t v[64];
+      if (active) {
+        tmem_ld32(tmem + lane_off + C::TM_DP + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + lane_off + C::TM_DP + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      }
+      tc_fence_before();
+      mbar_arrive(bars + 8 * (C::B_DQ_EMPTY + b));
+      // the staging buffer sb is free once the reduce issued NDQ tiles ago has read it
+      if (issuer) {
+        bulk_wait_read<C::NDQ - 1>();
+        mbar_arrive(bars + 8 * (C::B_STG_FREE + sb));
+      }
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (g / C::NDQ) & 1, BF_DR_FREE))))
+        break;
+      if (active) {
+        float* t = stg + sb * (C::DQ_TILE / 4) + c;
 #pragma unroll
-          for (int q = 0; q < C::BQ; ++q) t[q * D] = __uint_as_float(v[q]);
-        }
-      } else {
-        // staging buffer first, then 32 columns at a time through registers
-        // (fewer live registers), releasing the tensor-memory buffer after
-        if (issuer) {
-          bulk_wait_read<C::NDQ - 1>();
-          mbar_arrive(bars + 8 * (C::B_STG_FREE + sb));
-        }
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_STG_FREE + sb), (g / C::NDQ) & 1, BF_DR_FREE))))
-          break;
-        if (active) {
-          float* t = stg + sb * (C::DQ_TILE / 4) + c;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + C::TM_DP + b * 64 + h * 32, v);
-            tmem_ld_wait();
-            reg_fence(v);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) t[(h * 32 + q) * D] = __uint_as_float(v[q]);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bars + 8 * (C::B_DQ_EMPTY + b));
+        for (int q = 0; q < C::BQ; ++q) t[q * D] = __uint_as_float(v[q]);
       }
       fence_proxy_async_smem();
       mbar_arrive(bars + 8 * (C::B_STG_FULL + sb));
