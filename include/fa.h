@@ -251,6 +251,25 @@ const char* fa_fwd_kernel_name(int d, int causal);
 const char* fa_bwd_dkdv_kernel_name(int d);
 
 /*
+ * The per-CTA unit lists the causal kernels follow, for inspection and tests
+ * (host only: no GPU, no device call).  kind 0: the one-SM forward's lists
+ * (units = pairs of 128-row query tiles of a head; unit index r*B*H + bh is
+ * query-tile pair NP-1-r of head bh, NP = ceil(ceil(N/128)/2)), built for
+ * 128-key tiles; kind 1: the persistent fused backward's lists (units = 128-key
+ * tiles of a head, numbered in the kernel's grouped longest-first order).
+ * Lists hold each unit once: CTA c runs order[start[c] .. start[c+1]).
+ * `grid` CTAs (1 .. 160); `start` has room for grid + 1 entries, `order` for
+ * max_units.  Returns the number of units (the lists are written), 0 when the
+ * shape has no lists (more than 4096 units: the kernels deal the units in
+ * serpentine order instead; nothing is written), or FA_ERR_INVALID_ARG (bad
+ * kind, sizes or grid, or max_units too small).  The paper has no
+ * counterpart: this is how the kernels balance the causal mask's unequal
+ * units over the SMs.
+ */
+int fa_unit_lists(int kind, int B, int H, int N, int d, int grid, unsigned short* start, unsigned short* order,
+                  int max_units);
+
+/*
  * Fault-detection self test.  Launches one tiny kernel that waits on a
  * barrier nothing ever signals, with a wall-clock limit of `limit_us`
  * microseconds (1 .. 10,000,000).  The wait runs out, the kernel records

@@ -949,6 +949,22 @@ int heads_per_group(int BH, int groups) {
 }
 }  // namespace
 
+extern "C" int fa_unit_lists(int kind, int B, int H, int N, int d, int grid, unsigned short* start,
+                             unsigned short* order, int max_units) {
+  if ((kind != 0 && kind != 1) || check_sizes(B, H, N, d) || grid < 1 || grid > fa::UnitList::kMaxCtas || !start ||
+      !order)
+    return FA_ERR_INVALID_ARG;
+  const int BH = B * H;
+  fa::UnitList L;
+  L.n = 0;
+  const bool built = kind == 0 ? build_unit_list(&L, BH, N, d, 128, grid) : build_bwd_unit_list(&L, BH, N, d, grid);
+  if (!built) return 0;
+  if (max_units < L.n) return FA_ERR_INVALID_ARG;
+  for (int c = 0; c <= grid; ++c) start[c] = L.start[c];
+  for (int i = 0; i < L.n; ++i) order[i] = L.order[i];
+  return L.n;
+}
+
 extern "C" size_t fa_fwd_bwd_host_workspace_bytes(int B, int H, int N, int d, int groups) {
   if (check_sizes(B, H, N, d) || groups < 1) return 0;
   return kHostSlots * host_slot(heads_per_group(B * H, groups), N, d).total;

@@ -85,6 +85,8 @@ def load_library(build_if_missing: bool = True):
         lib.fa_bwd_set_phase_events.restype = None
         lib.fa_fwd_bwd_host_workspace_bytes.argtypes = [i, i, i, i, i]
         lib.fa_fwd_bwd_host_workspace_bytes.restype = sz
+        lib.fa_unit_lists.argtypes = [i, i, i, i, i, i, vp, vp, i]
+        lib.fa_unit_lists.restype = i
         lib.fa_fwd_bwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
         lib.fa_fwd_bwd_host.restype = i
         lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
@@ -273,6 +275,24 @@ def backward_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | N
 
 def host_workspace_bytes(B: int, H: int, N: int, d: int, groups: int) -> int:
     return int(load_library().fa_fwd_bwd_host_workspace_bytes(B, H, N, d, groups))
+
+
+def unit_lists(kind: int, B: int, H: int, N: int, d: int, grid: int):
+    """The causal kernels' per-CTA unit lists (fa_unit_lists; host only):
+    kind 0 the one-SM forward, 1 the persistent backward.  Returns a list of
+    `grid` lists of unit indices, or None when the shape has none (more units
+    than the lists hold: the kernels deal them in serpentine order)."""
+    lib = load_library()
+    max_units = 4096
+    start = (ctypes.c_ushort * (grid + 1))()
+    order = (ctypes.c_ushort * max_units)()
+    n = int(lib.fa_unit_lists(kind, B, H, N, d, grid, ctypes.cast(start, ctypes.c_void_p),
+                              ctypes.cast(order, ctypes.c_void_p), max_units))
+    if n < 0:
+        raise FaError(n, "fa_unit_lists")
+    if n == 0:
+        return None
+    return [list(order[start[c]:start[c + 1]]) for c in range(grid)]
 
 
 def _check_host(*ts):

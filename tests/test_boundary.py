@@ -26,7 +26,8 @@ def test_every_declared_symbol_is_exported(lib):
                           "fa_status_string", "fa_selftest_wait_timeout", "fa_bwd_set_phase_events",
                           "fa_last_cuda_error", "fa_bwd_noalloc", "fa_fwd_kernel_name",
                           "fa_fwd_unfused", "fa_fwd_unfused_workspace_bytes", "fa_bwd_dkdv_kernel_name",
-                          "fa_bwd_deterministic", "fa_fwd_bwd_host", "fa_fwd_bwd_host_workspace_bytes"}
+                          "fa_bwd_deterministic", "fa_fwd_bwd_host", "fa_fwd_bwd_host_workspace_bytes",
+                          "fa_unit_lists"}
     out = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (fa_\w+)", out))
     for n in names:
