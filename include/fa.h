@@ -90,8 +90,10 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *      bytes, 16-byte aligned, not overlapping any other argument; its
  *      contents on entry do not matter.
  * Three launches, in order on `stream`: the D = rowsum(dO * O) pass (which
- * also zeroes the dQ accumulator); fa_bwd_fused_kernel, one CTA per 128 keys
- * of a head, which recomputes P = exp(S - LSE) tile by tile and forms all
+ * also zeroes the dQ accumulator); fa_bwd_fused_kernel, persistent (one CTA
+ * per SM walking units of 128 keys of a head; with the mask each CTA's list
+ * of units is computed on the host at the first call for a shape and kept),
+ * which recomputes P = exp(S - LSE) tile by tile and forms all
  * five products of the gradient -- S, dP, dV, dK and the tile's share of dQ,
  * added into the fp32 accumulator by the bulk-copy engine; and a pass that
  * writes dQ = bf16(scale * accumulator).  dK and dV are accumulated in a
