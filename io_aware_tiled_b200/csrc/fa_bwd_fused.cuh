@@ -149,18 +149,7 @@ __device__ __forceinline__ void store_accumulator_row(uint32_t t_row, __nv_bfloa
     tmem_ld32(t_row + cc * 32, a);
     tmem_ld_wait();
     reg_fence(a);
-    if (valid) {
-      uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 wv;
-        wv.x = pack_bf16(__uint_as_float(a[8 * v + 0]) * mul, __uint_as_float(a[8 * v + 1]) * mul);
-        wv.y = pack_bf16(__uint_as_float(a[8 * v + 2]) * mul, __uint_as_float(a[8 * v + 3]) * mul);
-        wv.z = pack_bf16(__uint_as_float(a[8 * v + 4]) * mul, __uint_as_float(a[8 * v + 5]) * mul);
-        wv.w = pack_bf16(__uint_as_float(a[8 * v + 6]) * mul, __uint_as_float(a[8 * v + 7]) * mul);
-        dst[v] = wv;
-      }
-    }
+    if (valid) store_bf16x32(dst_row + cc * 32, a, mul);
   }
 }
 

@@ -679,6 +679,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 32 fp32 values (as raw bits) times `mul`, as 32 bf16 (64 bytes) at `dst`
+// (16-byte aligned): two 32-byte stores when `dst` is 32-byte aligned, so each
+// writes whole 32-byte sectors, else four 16-byte stores.
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&a)[32], float mul) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) w[i] = pack_bf16(__uint_as_float(a[2 * i]) * mul, __uint_as_float(a[2 * i + 1]) * mul);
+  if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 16), "r"(w[8]), "r"(w[9]),
+                 "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+                 : "memory");
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+  }
+}
+
 // Index of the k-th work unit of a persistent worker w out of W: units are
 // dealt in rounds of W, left to right on even rounds and right to left on odd
 // ones ("serpentine").  With units sorted longest first this balances the

@@ -542,18 +542,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
         tmem_ld32(tO + c * 32, o);
         tmem_ld_wait();
         reg_fence(o);
-        if (row < N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-            w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-            w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-            w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-            dst[v] = w;
-          }
-        }
+        if (row < N) store_bf16x32(orow + c * 32, o, inv_l);
       }
       if (row < N) LSE[static_cast<size_t>(bh) * N + row] = (m_ref + __log2f(l)) * kLn2;
       tc_fence_before();

@@ -290,6 +290,35 @@ def test_gradient_outputs_stay_inside_their_buffers():
         assert (b[:guard] == 3.5).all() and (b[guard + n:] == 3.5).all()
 
 
+def test_outputs_at_a_16_byte_offset():
+    """O, dK and dV are written with 32-byte stores when the row start is
+    32-byte aligned and with 16-byte stores otherwise (the ABI asks for 16-byte
+    alignment).  Outputs 8 elements (16 bytes) past a 32-byte boundary equal,
+    bit for bit, those written into aligned buffers, for every forward kernel
+    and the backward, and the guard elements around them stay untouched."""
+    dev = _dev()
+    for B, H, N, d, causal in ((1, 2, 300, 128, False), (1, 2, 300, 128, True), (1, 2, 300, 64, False)):
+        q, k, v, do = (t.to(dev) for t in attention_inputs(B, H, N, d, seed=41))
+        n = B * H * N * d
+        o_ref, lse = fa.forward(q, k, v, causal)
+        obuf = torch.full((n + 64,), -7.0, dtype=torch.bfloat16, device=dev)
+        o = obuf[8:8 + n].view(B, H, N, d)
+        assert o.data_ptr() % 32 == 16
+        fa.forward(q, k, v, causal, out=o, lse=torch.empty_like(lse))
+        assert fa.sync_status() == fa.FA_OK
+        assert torch.equal(o, o_ref), (B, H, N, d, causal)
+        assert (obuf[:8] == -7.0).all() and (obuf[8 + n:] == -7.0).all()
+        g_ref = fa.backward(q, k, v, o_ref, do, lse, causal)
+        bufs = [torch.full((n + 64,), 3.5, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        views = [b[8:8 + n].view(B, H, N, d) for b in bufs]
+        fa.backward(q, k, v, o_ref, do, lse, causal, dq=views[0], dk=views[1], dv=views[2])
+        assert fa.sync_status() == fa.FA_OK
+        assert torch.equal(views[1], g_ref[1]) and torch.equal(views[2], g_ref[2])
+        assert_same_up_to_summation_order(views[0], g_ref[0], "dQ at a 16-byte offset")
+        for b in bufs:
+            assert (b[:8] == 3.5).all() and (b[8 + n:] == 3.5).all()
+
+
 def test_forward_and_backward_are_deterministic():
     """The forward and the deterministic backward give identical bits on
     repeated calls.  The default backward gives identical dK and dV; its dQ
