@@ -339,22 +339,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
         }
         // a row whose keys so far are all masked keeps m = -inf and P = 0
         const float neg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // pairs of scores through the paired fp32 instructions (one FMA and one
+        // add for two elements); 4 x 2 independent partial row sums
+        const uint64_t sc2 = f2_make(scale_log2, scale_log2), ng2 = f2_make(neg, neg);
+        uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float t0 = fmaf(s[32 * ch + 2 * c], scale_log2, neg);
-            const float t1 = fmaf(s[32 * ch + 2 * c + 1], scale_log2, neg);
+            float t0, t1;
+            f2_split(f2_fma(f2_make(s[32 * ch + 2 * c], s[32 * ch + 2 * c + 1]), sc2, ng2), t0, t1);
             const bool emul = c % C::EXP_EMUL_EVERY == C::EXP_EMUL_EVERY - 1;  // resolved at compile time
             const float p0 = emul ? exp2_poly3(t0) : ex2(t0);
             const float p1 = emul ? exp2_poly3(t1) : ex2(t1);
-            ps[c & 7] += p0 + p1;
+            ps2[c & 3] = f2_add(ps2[c & 3], f2_make(p0, p1));
             p[c] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + 32 * h + ch * 16, p);  // keys 64h.. -> packed columns 32h..
         }
+        float ps[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f2_split(ps2[e], ps[2 * e], ps[2 * e + 1]);
 #pragma unroll
         for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
