@@ -695,6 +695,32 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return r;
 }
 
+// exp2_poly3 of the two values of a pair, on the paired fp32 instructions:
+// the same operations lane by lane (the same results), half the FMA-pipe
+// instructions.
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ void exp2_poly3_x2(uint64_t t2, float& p0, float& p1) {
+  float t0, t1;
+  f2_split(t2, t0, t1);
+  const uint64_t t = f2_make(fmaxf(t0, -126.f), fmaxf(t1, -126.f));
+  const uint64_t magic = f2_make(12582912.f, 12582912.f);
+  const uint64_t r = f2_add(t, magic);
+  const uint64_t f = f2_sub(t, f2_sub(r, magic));
+  const uint64_t c3 = f2_make(0.05517166853f, 0.05517166853f), c2 = f2_make(0.2426111251f, 0.2426111251f);
+  const uint64_t c1 = f2_make(0.6932609677f, 0.6932609677f), c0 = f2_make(0.9999280572f, 0.9999280572f);
+  const uint64_t p = f2_fma(f2_fma(f2_fma(c3, f, c2), f, c1), f, c0);
+  float q0, q1, r0, r1;
+  f2_split(p, q0, q1);
+  f2_split(r, r0, r1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(r0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(r1) << 23));
+}
+
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
   return *reinterpret_cast<uint32_t*>(&v);

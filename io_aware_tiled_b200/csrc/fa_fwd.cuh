@@ -489,11 +489,16 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
           uint32_t p[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            float t0, t1;
-            f2_split(f2_fma(f2_make(s[32 * ch + 2 * c], s[32 * ch + 2 * c + 1]), sc2, ng2), t0, t1);
-            const bool emul = c % C::EXP_EMUL_EVERY == C::EXP_EMUL_EVERY - 1;  // resolved at compile time
-            const float p0 = emul ? exp2_poly3(t0) : ex2(t0);
-            const float p1 = emul ? exp2_poly3(t1) : ex2(t1);
+            const uint64_t t2 = f2_fma(f2_make(s[32 * ch + 2 * c], s[32 * ch + 2 * c + 1]), sc2, ng2);
+            float p0, p1;
+            if (c % C::EXP_EMUL_EVERY == C::EXP_EMUL_EVERY - 1) {  // resolved at compile time
+              exp2_poly3_x2(t2, p0, p1);
+            } else {
+              float t0, t1;
+              f2_split(t2, t0, t1);
+              p0 = ex2(t0);
+              p1 = ex2(t1);
+            }
             ps2[c & 3] = f2_add(ps2[c & 3], f2_make(p0, p1));
             p[c] = pack_bf16(p0, p1);
           }

@@ -68,3 +68,22 @@ def test_masked_scores_give_tiny_nonnegative_values():
     p = np.float32(c[0])  # f = 0
     wrapped = (np.array([p]).view(np.int32) + (r.view(np.int32) << 23)).view(np.float32)
     assert np.isnan(wrapped).all()
+
+
+def test_paired_form_uses_the_same_steps():
+    """exp2_poly3_x2 (two values on the paired fp32 instructions) repeats the
+    scalar form's clamp, rounding constant and polynomial lane by lane."""
+    src = open(os.path.join(CSRC, "fa_device.cuh"), encoding="utf-8").read()
+    body = src[src.index("void exp2_poly3_x2("):]
+    body = body[:body.index("\n}\n")]
+    clamp, c = _kernel_constants()
+    assert body.count(f"fmaxf(t0, {clamp:.0f}.f)") == 1 and body.count(f"fmaxf(t1, {clamp:.0f}.f)") == 1
+    pairs = re.findall(r"f2_make\(([0-9.e-]+)f, ([0-9.e-]+)f\)", body)
+    vals = {float(a) for a, b in pairs if a == b}
+    assert all(a == b for a, b in pairs)
+    assert 12582912.0 in vals
+    for k in range(4):
+        assert any(np.float32(v) == c[k] for v in vals), c[k]
+    assert "f2_fma(f2_fma(f2_fma(c3, f, c2), f, c1), f, c0)" in body
+    scalar = src[src.index("float exp2_poly3(float t)"):]
+    assert "12582912.f" in scalar[:scalar.index("}")]
