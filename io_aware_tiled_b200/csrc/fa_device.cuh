@@ -694,6 +694,22 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Multiply 32 fp32 values (raw bits, in place) by `mul`, two per instruction.
+__device__ __forceinline__ void scale32(uint32_t (&a)[32], float mul) {
+  const uint64_t m2 = f2_make(mul, mul);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float lo, hi;
+    f2_split(f2_mul(f2_make(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), m2), lo, hi);
+    a[2 * i] = __float_as_uint(lo);
+    a[2 * i + 1] = __float_as_uint(hi);
+  }
+}
 
 // exp2_poly3 of the two values of a pair, on the paired fp32 instructions:
 // the same operations lane by lane (the same results), half the FMA-pipe
@@ -731,8 +747,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // writes whole 32-byte sectors, else four 16-byte stores.
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&a)[32], float mul) {
   uint32_t w[16];
+  const uint64_t m2 = f2_make(mul, mul);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) w[i] = pack_bf16(__uint_as_float(a[2 * i]) * mul, __uint_as_float(a[2 * i + 1]) * mul);
+  for (int i = 0; i < 16; ++i) {  // two products per paired multiply
+    float lo, hi;
+    f2_split(f2_mul(f2_make(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), m2), lo, hi);
+    w[i] = pack_bf16(lo, hi);
+  }
   if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
     asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
                  "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])

@@ -529,8 +529,7 @@ __global__ void __launch_bounds__(FwdCfg<D, BN_>::THREADS, 1)
             tmem_ld32(tO + c * 32, o);
             tmem_ld_wait();
             reg_fence(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            scale32(o, alpha);
             tmem_st32(tO + c * 32, o);
           }
         }
