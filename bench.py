@@ -305,14 +305,14 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
     # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal_dram.md (32 heads)
-    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.752896e6 + 14.989056e6) / 32,
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.752128e6 + 16.377856e6) / 32,
                           "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "f428f9dfcfe88488595cb49ee7e0cda682e39970c17846694a8c9bfe4cdb5b5b"},
+                          "sha256": "ca851025911bb96e321d41ec1ffef4606d93862cf5886f78c3b3ac1a888a1ee5"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
-    "fa_bwd_fused_kernel": {"bytes_per_head": (202.483968e6 + 84.928e6) / 32,
+    "fa_bwd_fused_kernel": {"bytes_per_head": (202.500608e6 + 88.388096e6) / 32,
                             "sources": ("fa_bwd_fused.cuh", "fa_device.cuh"),
-                            "sha256": "105bf34fac7f3c4da0ff73015c2bd47077d6590b103b4b4fd380f32faddc2c1f"},
+                            "sha256": "02792bfbc6b93aa187de7a59b1202e51558a2fa39f2366c72cd879a7c40c0d59"},
 }
 
 
