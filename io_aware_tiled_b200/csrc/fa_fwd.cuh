@@ -36,11 +36,16 @@
 //     and PV-count parity).
 //   * Softmax: each thread owns one full row of S (tcgen05.ld 32x32b), so the
 //     row max and row sum are register reductions.  Work is in base 2 with
-//     scale*log2(e) folded into one FMA.  O is rescaled only when a row's max
-//     grows by more than a factor 2^rescale_log2 (8 by default; exact: the
-//     final division uses the same max).  A fixed share of the exponentials
-//     runs on the FMA pipe (exp2_poly3), the rest on the MUFU.
-//   * Epilogue: O / l as bf16 and LSE as fp32, stored once per row.
+//     scale*log2(e) folded into one FMA, issued for two scores at a time
+//     (fma.rn.f32x2; the row sum and the O rescale use the paired add and
+//     multiply too).  O is rescaled only when a row's max grows by more than
+//     a factor 2^rescale_log2 (8 by default; exact: the final division uses
+//     the same max).  A fixed share of the exponentials runs on the FMA pipe
+//     (exp2_poly3_x2, two at a time), the rest on the MUFU.
+//   * Epilogue: O / l as bf16 and LSE as fp32, stored once per row (32-byte
+//     stores where the rows are 32-byte aligned).
+//   * With one Q buffer (d = 128) a unit's Q pair is released after its last
+//     S product, so the next unit's Q loads while its last PVs run.
 #pragma once
 
 #include "fa_device.cuh"

@@ -28,7 +28,11 @@
 //     the columns) is rescaled only when a row max grows by more than a factor
 //     2^rescale_log2 (8 by default), after waiting for the previous PV (an "O
 //     done" barrier committed after every PV).  One exponential in 8 runs on
-//     the FMA pipe (exp2_poly3).
+//     the FMA pipe (exp2_poly3).  The exponent arguments, the row sums and the
+//     O rescale use the paired fp32 instructions (two values per instruction).
+//   * A unit's Q tiles are released after its last S product, so the next
+//     unit's Q loads while its last PVs run; the leader waits for the last
+//     PV's V_EMPTY arrival before the teardown.
 #pragma once
 
 #include "fa_device.cuh"
