@@ -307,7 +307,7 @@ NCU_TRAFFIC = {
     # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal_dram.md (32 heads)
     "fa_fwd_2sm_kernel": {"bytes_per_head": (100.752128e6 + 16.377856e6) / 32,
                           "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "ca851025911bb96e321d41ec1ffef4606d93862cf5886f78c3b3ac1a888a1ee5"},
+                          "sha256": "1de9828655fbfa75df16476a61ae9641f78ba8a8f44e5f69c78b35bd591f95a5"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
     "fa_bwd_fused_kernel": {"bytes_per_head": (202.500608e6 + 88.388096e6) / 32,
