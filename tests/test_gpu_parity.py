@@ -246,6 +246,17 @@ def test_workload_long_b1h16n16384d128():
     _full_backward_check(w, True, q, k, v, do, o, lse, heads=[0, 15], n_rows=256)
 
 
+def test_longer_than_every_workload():
+    """N = 32768 (twice the long workload; 1024 query tiles of the backward, 256
+    key tiles per head): the forward with and without the mask on sampled
+    rows, the backward with the mask on sampled rows of both heads."""
+    from io_aware_tiled_b200.configs import Workload
+    w = Workload("longer_b1h2n32768d128", 1, 2, 32768, 128, (False, True), True)
+    _full_forward_check(w, False, heads_full=[], n_random_rows=96)
+    q, k, v, do, o, lse = _full_forward_check(w, True, heads_full=[], n_random_rows=96)
+    _full_backward_check(w, True, q, k, v, do, o, lse, heads=[0, 1], n_rows=48)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_workload_ragged_b8h12n1000d64(causal):
     w = WORKLOADS["ragged_b8h12n1000d64"]
