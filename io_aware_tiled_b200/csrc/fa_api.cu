@@ -293,7 +293,7 @@ float effective_scale(float scale, int d, bool* ok) {
 // Unit lists of the causal one-SM forward.  A unit is a pair of 128-row query
 // tiles of one head; pair p of a head runs (2p+1) + (2p+2) key-tile steps
 // (scaled by 128 / BN), plus about one step per query tile of fixed cost.
-// Order: heads in groups whose K and V fit in 64 MiB of L2, inside a group the
+// Order: heads in groups whose K and V fit in 32 MiB of L2, inside a group the
 // longest units first; then a longest-processing-time assignment: each unit
 // in that order goes to the CTA with the least work so far.  Each CTA runs its
 // units in assignment order.  Lists are cached per shape (they depend only on
@@ -307,7 +307,7 @@ UnitListEntry g_lists[kListCache];
 int g_lists_next = 0;
 std::mutex g_lists_mu;
 
-constexpr long long kFwdGroupBytes = 64ll << 20;  // K and V of a head group
+constexpr long long kFwdGroupBytes = 32ll << 20;  // K and V of a head group
 
 // Longest-processing-time assignment of units, taken in the given order (the
 // caller puts the longest first), each to the CTA with the least work so far;
