@@ -371,7 +371,7 @@ bool causal_unit_list(fa::FwdUnitList* out, int BH, int N, int d, int bn, int gr
 
 // Unit lists of the persistent fused backward with the mask.  Unit u is key
 // tile kt of head bh in the kernel's grouped order (heads in groups whose K
-// and V fit in 64 MiB of L2, the first key tiles -- those that see the most
+// and V fit in 32 MiB of L2, the first key tiles -- those that see the most
 // query tiles -- first); its cost is its query tiles plus one for the unit's
 // fixed work (K and V loads, the dK and dV stores, mostly overlapped).
 UnitListEntry g_bwd_lists[kListCache];

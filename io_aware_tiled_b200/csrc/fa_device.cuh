@@ -779,11 +779,11 @@ __device__ __forceinline__ int serpentine_unit(int k, int w, int W) {
 // Causal block orders of the backward launch the longest blocks first so the
 // last wave is short; across all heads at once, that keeps every head's K and
 // V (or Q and dO) in flight.  Heads therefore go in groups whose K and V
-// (bf16) fit in 64 MiB of the 126 MB L2 (all heads when they fit), longest
+// (bf16) fit in 32 MiB of the 126 MB L2 (all heads when they fit), longest
 // blocks first inside each group.  Returns the group size.
 __host__ __device__ __forceinline__ int causal_head_group(int BH, int N, int D) {
   const long long per_head = 4ll * N * D;
-  const long long g = (64ll << 20) / per_head;
+  const long long g = (32ll << 20) / per_head;
   return g >= BH ? BH : (g < 1 ? 1 : static_cast<int>(g));
 }
 // Unit u of that order for units of NR ranks per head (rank 0 = longest):

@@ -10,7 +10,7 @@ from io_aware_tiled_b200 import fa
 EINVAL = -1
 SMS = 148
 FWD_GROUP_BYTES = 32 << 20  # K and V of a head group kept in L2: the forward's lists
-BWD_GROUP_BYTES = 64 << 20  # and the backward's
+BWD_GROUP_BYTES = 32 << 20  # and the backward's
 
 
 def _group(BH, N, d, group_bytes):
