@@ -60,8 +60,9 @@ typedef enum {
  * Out: O [B,H,N,d] bf16 (O = P V, rounded to nearest even), LSE [B,H,N] fp32.
  * One persistent kernel launch on `stream`: CTA pairs (fa_fwd_2sm_kernel) for
  * d = 128 without the mask, one SM per CTA (fa_fwd_kernel) otherwise.  With
- * the mask the launch carries each CTA's list of query-tile pairs, computed on
- * the host at the first call for a shape and kept (a few shapes at a time).  Two
+ * the mask the launch carries each CTA's (the paired kernel: each CTA pair's)
+ * list of query-tile pairs, computed on the host at the first call for a
+ * shape and kept (a few shapes at a time).  Two
  * environment variables, read at each call, select other forms for
  * comparisons: FA_FWD_PAIR=0 / =1 forces the one-SM / paired kernel for
  * d = 128; FA_FWD_BN=64 runs the one-SM kernel with 64-key K/V tiles instead
@@ -254,7 +255,8 @@ const char* fa_bwd_dkdv_kernel_name(int d);
 
 /*
  * The per-CTA unit lists the causal kernels follow, for inspection and tests
- * (host only: no GPU, no device call).  kind 0: the one-SM forward's lists
+ * (host only: no GPU, no device call).  kind 0: the causal forward's lists
+ * (grid = CTAs of the one-SM kernel, or CTA pairs of the paired kernel)
  * (units = pairs of 128-row query tiles of a head; unit index r*B*H + bh is
  * query-tile pair NP-1-r of head bh, NP = ceil(ceil(N/128)/2)), built for
  * 128-key tiles; kind 1: the persistent fused backward's lists (units = 128-key

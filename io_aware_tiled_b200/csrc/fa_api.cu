@@ -500,10 +500,14 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
     const float sl2p = sc * fa::kLog2e;
     cudaStream_t sp = static_cast<cudaStream_t>(stream);
     auto* op = static_cast<__nv_bfloat16*>(O);
-    if (causal)
-      fa::fa_fwd_2sm_kernel<true><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p, rescale);
-    else
-      fa::fa_fwd_2sm_kernel<false><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p, rescale);
+    if (causal) {
+      fa::FwdUnitList pl;  // per CTA pair (n = 0: serpentine deal)
+      pl.n = 0;
+      causal_unit_list(&pl, BH, N, d, 128, pairs);
+      fa::fa_fwd_2sm_kernel<true><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p, rescale, pl);
+    } else {
+      fa::fa_fwd_2sm_kernel<false><<<2 * pairs, fa::Fwd2Cfg::THREADS, fa::Fwd2Cfg::SMEM_BYTES, sp>>>(mq, mkh, mv, op, LSE, BH, N, sl2p, rescale, fa::FwdNoList{0});
+    }
     return launch_status();
   }
   const int nqt = (N + 127) / 128, units = BH * ((nqt + 1) / 2);

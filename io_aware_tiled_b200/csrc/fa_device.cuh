@@ -819,17 +819,22 @@ struct UnitListOf<true> {
   using type = UnitList;
 };
 
-// The k-th unit of this CTA in `list` (>= units when it has no more); without
-// a list, the units dealt in serpentine order over the grid.
+// The k-th unit of worker w (of W) in `list` (>= units when it has no more);
+// without a list, the units dealt in serpentine order over the W workers.
 template <typename L>
-__device__ __forceinline__ int list_unit(const L& list, int k, int units) {
+__device__ __forceinline__ int worker_unit(const L& list, int k, int units, int w, int W) {
   if constexpr (sizeof(L) > sizeof(NoUnitList)) {
     if (list.n > 0) {
-      const int i = list.start[blockIdx.x] + k;
-      return i < list.start[blockIdx.x + 1] ? static_cast<int>(list.order[i]) : units;
+      const int i = list.start[w] + k;
+      return i < list.start[w + 1] ? static_cast<int>(list.order[i]) : units;
     }
   }
-  return serpentine_unit(k, blockIdx.x, gridDim.x);
+  return serpentine_unit(k, w, W);
+}
+// The same with one worker per CTA.
+template <typename L>
+__device__ __forceinline__ int list_unit(const L& list, int k, int units) {
+  return worker_unit(list, k, units, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

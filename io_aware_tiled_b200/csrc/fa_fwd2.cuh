@@ -76,8 +76,11 @@ enum Fwd2WaitSite : unsigned int {
 };
 
 // Pair unit u covers query tiles 2*qp (rank 0) and 2*qp+1 (rank 1) of head bh.
-// Non-causal: head-major (concurrent pairs share a few heads' K/V in L2).
-// Causal: longest units first across all heads.
+// Non-causal: head-major (concurrent pairs share a few heads' K/V in L2),
+// dealt in serpentine order.  Causal: numbered longest first across all
+// heads; the host's per-pair lists (the one-SM kernel's unit lists, one
+// worker per CTA pair: heads in L2-sized groups, longest first inside a
+// group, longest-processing-time assignment) say which pair runs which.
 __device__ __forceinline__ void fwd2_decode_unit(int u, int BH, int NQP, bool causal, int& bh, int& qp) {
   if (causal) {
     const int r = u / BH;
@@ -93,8 +96,8 @@ template <bool CAUSAL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     fa_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKh,
                       const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-                      float* __restrict__ LSE, int BH, int N, float scale_log2,
-                  float rescale_log2) {
+                      float* __restrict__ LSE, int BH, int N, float scale_log2, float rescale_log2,
+                      const __grid_constant__ typename UnitListOf<CAUSAL>::type list) {
   using C = Fwd2Cfg;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -157,7 +160,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     // ------------------------------------------------------------ loads (both CTAs)
     if (lane == 0) {
       uint32_t kv_it = 0, q_it = 0;
-      for (int k = 0, u = pair; u < units; u = serpentine_unit(++k, pair, npairs)) {
+      for (int k = 0, u = worker_unit(list, 0, units, pair, npairs); u < units; u = worker_unit(list, ++k, units, pair, npairs)) {
         int bh, qp;
         fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
         const int nk = CAUSAL ? min(2 * qp + 2, NKT) : NKT;
@@ -206,7 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
       tc_commit_pair_warp(bar(C::B_K_EMPTY + s), C::BOTH);
       return true;
     };
-    for (int k = 0, u = pair; u < units && ok; u = serpentine_unit(++k, pair, npairs), ++unit_it) {
+    for (int k = 0, u = worker_unit(list, 0, units, pair, npairs); u < units && ok; u = worker_unit(list, ++k, units, pair, npairs), ++unit_it) {
       int bh, qp;
       fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
       (void)bh;
@@ -258,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     // leader's, one remote arrival per phase.
     if (lane == 0) {
       uint32_t g = 0, unit_it = 0;
-      for (int k = 0, u = pair; u < units; u = serpentine_unit(++k, pair, npairs), ++unit_it) {
+      for (int k = 0, u = worker_unit(list, 0, units, pair, npairs); u < units; u = worker_unit(list, ++k, units, pair, npairs), ++unit_it) {
         int bh, qp;
         fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
         (void)bh;
@@ -290,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fwd2Cfg::THREADS, 1)
     float* xsum = xch + 4 * 128;              // [half][row]
     uint32_t s_it = 0;
     bool ok = true;
-    for (int k = 0, u = pair; u < units && ok; u = serpentine_unit(++k, pair, npairs)) {
+    for (int k = 0, u = worker_unit(list, 0, units, pair, npairs); u < units && ok; u = worker_unit(list, ++k, units, pair, npairs)) {
       int bh, qp;
       fwd2_decode_unit(u, BH, NQP, CAUSAL, bh, qp);
       const int qt = 2 * qp + static_cast<int>(rank);

@@ -88,6 +88,19 @@ def test_forward_lists(B, H, N, d):
         assert ratio <= 1.04, ratio
 
 
+@pytest.mark.parametrize("B,H,N,d", [s for s in SHAPES if s[3] == 128])
+def test_forward_lists_per_cta_pair(B, H, N, d):
+    """The paired (two-SM) kernel's lists with the mask: the same units and
+    builder, one worker per CTA pair (74 pairs on 148 SMs)."""
+    BH = B * H
+    cost = _fwd_units(BH, N)
+    grid = min(len(cost), SMS // 2)
+    lists = fa.unit_lists(0, B, H, N, d, grid)
+    ratio = _check(lists, cost, _fwd_position(BH, N, d), grid)
+    if len(cost) >= 6 * grid:
+        assert ratio <= 1.04, ratio
+
+
 @pytest.mark.parametrize("B,H,N,d", SHAPES)
 def test_backward_lists(B, H, N, d):
     BH = B * H
