@@ -305,14 +305,14 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
     # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal_dram.md (32 heads)
-    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.788736e6 + 16.937728e6) / 32,
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.786432e6 + 16.232704e6) / 32,
                           "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "843238fbcba64401179b624f3f0fa9a7f34891548cd4f30204aed51ab5f73dfc"},
+                          "sha256": "20522d634199f7819a0976e63f46e1f3b7a9cc962d395dc016e6bb1d34e8242b"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
-    "fa_bwd_fused_kernel": {"bytes_per_head": (202.669312e6 + 88.374272e6) / 32,
+    "fa_bwd_fused_kernel": {"bytes_per_head": (202.783232e6 + 89.071104e6) / 32,
                             "sources": ("fa_bwd_fused.cuh", "fa_device.cuh"),
-                            "sha256": "c7201b00db4d82f73ea162d244458eec30e610d5ec7c3abc81702c163e9452bd"},
+                            "sha256": "10712ac827f60ff9c1f3d904fe9983ede338e21f9f2f431e7457112fe01cab32"},
 }
 
 
