@@ -463,6 +463,36 @@ def test_both_forward_kernels_for_d128(B, H, N, causal, monkeypatch):
     monkeypatch.delenv("FA_FWD_PAIR")
 
 
+def test_paired_forward_walks_every_unit_with_the_mask(monkeypatch):
+    """With the mask the paired kernel follows per-pair unit lists (at most
+    4096 units; beyond, a serpentine deal).  Shapes with several units per
+    CTA pair, on the lists and past them: sampled heads, from both ends of
+    every batch, match the oracle; every head's LSE matches the one-SM
+    kernel's to rounding, so no unit was skipped or run twice."""
+    dev = _dev()
+    monkeypatch.setenv("FA_FWD_PAIR", "1")
+    assert fa.forward_kernel_name(128, True) == "fa_fwd_2sm_kernel"
+    d = 128
+    for B, H, N in ((2, 40, 1000), (4, 300, 2048)):   # 320 units on the lists; 9600, past them
+        q, k, v, _ = attention_inputs(B, H, N, d, seed=51 + N, with_do=False)
+        qd, kd, vd = (t.to(dev) for t in (q, k, v))
+        o, lse = fa.forward(qd, kd, vd, True)
+        assert fa.sync_status() == fa.FA_OK
+        monkeypatch.setenv("FA_FWD_PAIR", "0")
+        _, lse1 = fa.forward(qd, kd, vd, True)
+        assert fa.sync_status() == fa.FA_OK
+        monkeypatch.setenv("FA_FWD_PAIR", "1")
+        assert (lse - lse1).abs().max().item() <= 1e-3, f"{B,H,N} LSE of the two kernels"
+        for b, h in ((0, 0), (B - 1, H - 1), (B // 2, H // 2)):
+            ro, rl = oracle.forward(f64(q[b:b + 1, h:h + 1]), f64(k[b:b + 1, h:h + 1]), f64(v[b:b + 1, h:h + 1]),
+                                    True, 1 / d ** 0.5)
+            what = f"paired {B,H,N} causal head {b},{h}"
+            check_o(f64(o[b:b + 1, h:h + 1].cpu()), ro, what)
+            check_lse(f64(lse[b:b + 1, h:h + 1].cpu()), rl, what)
+        del qd, kd, vd, o, lse, lse1
+    monkeypatch.delenv("FA_FWD_PAIR")
+
+
 def test_forward_kernel_name_follows_the_routing(monkeypatch):
     """fa_fwd_kernel_name reports the kernel fa_fwd launches: CTA pairs for
     d = 128 without the mask, one SM per CTA otherwise, FA_FWD_PAIR forcing
