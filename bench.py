@@ -304,10 +304,10 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # sha256 of the sources the kernel is compiled from at capture time: once they
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
-    # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal_dram.md (32 heads)
-    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.786432e6 + 16.232704e6) / 32,
+    # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal.md (32 heads)
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.751104e6 + 16.660736e6) / 32,
                           "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "20522d634199f7819a0976e63f46e1f3b7a9cc962d395dc016e6bb1d34e8242b"},
+                          "sha256": "5f41875604897ccbbd3527afe78924e4c9a70f37a3d9e2517cfb9d5d3941c3c2"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
     "fa_bwd_fused_kernel": {"bytes_per_head": (202.783232e6 + 89.071104e6) / 32,

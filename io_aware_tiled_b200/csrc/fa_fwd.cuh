@@ -92,8 +92,9 @@ struct FwdCfg {
   static constexpr uint32_t REGS_CONTROL = 64, REGS_SOFTMAX = 208;
   // one exponential pair in EXP_EMUL_EVERY goes to exp2_poly3 (FMA pipe)
   // instead of the MUFU: 1/16 of them at d = 64 (with the S ring the
-  // softmax's issue slots, not the MUFU, bound it), 1/8 at d = 128 (measured best)
-  static constexpr int EXP_EMUL_EVERY = (D == 64) ? 16 : 8;
+  // softmax's issue slots, not the MUFU, bound it), 1/4 at d = 128 (measured
+  // best under sustained load at the power limit, and no worse in isolated calls)
+  static constexpr int EXP_EMUL_EVERY = (D == 64) ? 16 : 4;
 };
 
 // wait-site identifiers recorded in the error word
