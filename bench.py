@@ -310,9 +310,9 @@ NCU_TRAFFIC = {
                           "sha256": "5f41875604897ccbbd3527afe78924e4c9a70f37a3d9e2517cfb9d5d3941c3c2"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
-    "fa_bwd_fused_kernel": {"bytes_per_head": (202.783232e6 + 89.071104e6) / 32,
+    "fa_bwd_fused_kernel": {"bytes_per_head": (202.964992e6 + 91.349248e6) / 32,
                             "sources": ("fa_bwd_fused.cuh", "fa_device.cuh"),
-                            "sha256": "10712ac827f60ff9c1f3d904fe9983ede338e21f9f2f431e7457112fe01cab32"},
+                            "sha256": "9759a63692390608395b1f568300fbe91584456129788f8fa122e098c86f7282"},
 }
 
 

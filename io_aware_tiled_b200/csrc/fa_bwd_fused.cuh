@@ -38,7 +38,7 @@
 //   warp 0       TMA: per unit the first ST query tiles (Q and dO, through ST
 //                stages), then K and V once the previous unit's products are
 //                done reading them, then the remaining query tiles;
-//                LSE*log2(e) and D of each query tile into shared memory.
+//                -LSE*log2(e) and D of each query tile into shared memory.
 //   warp 1       tcgen05.mma issue (one elected lane), commits; a unit's
 //                first dV and dK wait until the previous unit's are stored.
 //   warps 4-7    softmax gradient: thread = key row.  Reads S^T and dP^T
@@ -85,7 +85,7 @@ struct FusedCfg {
   static constexpr int OFF_DO = OFF_Q + ST * Q_TILE;
   static constexpr int OFF_DS = OFF_DO + ST * Q_TILE;
   static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;
-  static constexpr int OFF_LSE = OFF_DQ + NDQ * DQ_TILE;  // ST x BQ floats (LSE * log2 e)
+  static constexpr int OFF_LSE = OFF_DQ + NDQ * DQ_TILE;  // ST x BQ floats (-LSE * log2 e)
   static constexpr int OFF_DD = OFF_LSE + ST * BQ * 4;    // ST x BQ floats (D)
   static constexpr int OFF_BAR = OFF_DD + ST * BQ * 4;
   static constexpr int B_KV_FULL = 0, B_Q_FULL = 1, B_Q_EMPTY = 1 + ST, B_S_FULL = 1 + 2 * ST,
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
           for (int e = lane; e < C::BQ; e += 32) {
             const int q = qi * C::BQ + e;
             const bool valid = q < N;
-            sLSE[st * C::BQ + e] = valid ? LSE[static_cast<size_t>(bh) * N + q] * kLog2e : INFINITY;
+            sLSE[st * C::BQ + e] = valid ? -(LSE[static_cast<size_t>(bh) * N + q] * kLog2e) : -INFINITY;
             sDD[st * C::BQ + e] = valid ? Dvec[static_cast<size_t>(bh) * N + q] : 0.f;
           }
           mbar_arrive(bars + 8 * (C::B_Q_FULL + st));
@@ -375,7 +375,8 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
       reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
       reg_fence(*reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-      const float* lse2 = sLSE + st * C::BQ;
+      const float* nlse2 = sLSE + st * C::BQ;  // -LSE * log2(e) of the tile's queries
+      [[maybe_unused]] const uint64_t sc2 = f2_make(scale_log2, scale_log2);
       const float* dd = sDD + st * C::BQ;
       // masking: queries e < lim of this tile get P = 0 in this key row -- the
       // causal mask (query q sees key j iff j <= q) and key rows past N
@@ -389,14 +390,32 @@ __global__ void __launch_bounds__(FusedCfg<D, ST_, NDQ_>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const int e = 32 * ch + 2 * c;
-          float p0 = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, -lse2[e]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), scale_log2, -lse2[e + 1]));
+          // the same operations either way (one rounding per fma, sub, mul);
+          // at d = 64 on paired fp32 instructions, which measured faster there
+          // (at d = 128 the scalar form measured as fast or faster)
+          float p0, p1, ds0, ds1;
+          if constexpr (D == 64) {
+            f2_split(f2_fma(f2_make(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2,
+                            f2_make(nlse2[e], nlse2[e + 1])),
+                     p0, p1);
+          } else {
+            p0 = fmaf(__uint_as_float(sr[e]), scale_log2, nlse2[e]);
+            p1 = fmaf(__uint_as_float(sr[e + 1]), scale_log2, nlse2[e + 1]);
+          }
+          p0 = ex2(p0);
+          p1 = ex2(p1);
           if (mask) {
             if (e < lim) p0 = 0.f;
             if (e + 1 < lim) p1 = 0.f;
           }
-          const float ds0 = p0 * (__uint_as_float(dr[e]) - dd[e]);
-          const float ds1 = p1 * (__uint_as_float(dr[e + 1]) - dd[e + 1]);
+          if constexpr (D == 64) {
+            f2_split(f2_mul(f2_make(p0, p1), f2_sub(f2_make(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                                    f2_make(dd[e], dd[e + 1]))),
+                     ds0, ds1);
+          } else {
+            ds0 = p0 * (__uint_as_float(dr[e]) - dd[e]);
+            ds1 = p1 * (__uint_as_float(dr[e + 1]) - dd[e + 1]);
+          }
           pp[c] = pack_bf16(p0, p1);
           dsp[c] = pack_bf16(ds0, ds1);
         }
