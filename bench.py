@@ -460,12 +460,13 @@ def run_ours(args, rank, world, local_rank):
 
     from io_aware_tiled_b200.host_pipeline import forward_backward_host
 
-    ws_host = torch.empty(fa.host_workspace_bytes(B, H, N, d, 8), dtype=torch.uint8, device=dev)
+    E2E_GROUPS = 12  # head groups of the host pipeline (ceil(B*H / 12) heads each)
+    ws_host = torch.empty(fa.host_workspace_bytes(B, H, N, d, E2E_GROUPS), dtype=torch.uint8, device=dev)
 
     def e2e_pipelined():
         # fa_fwd_bwd_host: heads in groups through the library's three streams
         # (copies in, kernels, copies out)
-        forward_backward_host(hq, hk, hv, hdo, False, groups=8, out=(ho, hl, hdq, hdk, hdv), workspace=ws_host,
+        forward_backward_host(hq, hk, hv, hdo, False, groups=E2E_GROUPS, out=(ho, hl, hdq, hdk, hdv), workspace=ws_host,
                               device=dev)
 
     e2e_steps = max(3, args.steps // 4)
