@@ -305,9 +305,9 @@ def rank_seed(base_seed: int, rank: int) -> int:
 # change, the figure no longer describes the kernel and traffic is null.
 NCU_TRAFFIC = {
     # profiles/fa_fwd_2sm_kernel_b2h16n4096d128_noncausal.md (32 heads)
-    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.751104e6 + 16.660736e6) / 32,
+    "fa_fwd_2sm_kernel": {"bytes_per_head": (100.750592e6 + 20.326656e6) / 32,
                           "sources": ("fa_fwd2.cuh", "fa_device.cuh"),
-                          "sha256": "5f41875604897ccbbd3527afe78924e4c9a70f37a3d9e2517cfb9d5d3941c3c2"},
+                          "sha256": "79c9202b8bbf5a514ac67496b988089d804e0f304b16f3a083d27b3635801ac4"},
     # B=2, H=16, N=4096, d=128 non-causal (the bench's own shape, 32 heads):
     # profiles/fa_bwd_fused_kernel_b2h16n4096d128_noncausal.md
     "fa_bwd_fused_kernel": {"bytes_per_head": (202.964992e6 + 91.349248e6) / 32,

@@ -67,7 +67,7 @@ struct Fwd2Cfg {
   // warp 0 loads, warp 1 MMA (leader) or relay (peer), warps 4-7 and 8-11: the
   // softmax warpgroups of the low and the high 64 columns
   static constexpr int THREADS = 384;
-  static constexpr int EXP_EMUL_EVERY = 6;  // 1/6 of the exponentials on the FMA pipe (exp2_poly3)
+  static constexpr int EXP_EMUL_EVERY = 5;  // 1/5 of the exponentials on the FMA pipe (exp2_poly3)
   static constexpr uint16_t BOTH = 0x3;          // multicast mask: both CTAs of the pair
 };
 
